@@ -1,0 +1,416 @@
+#!/usr/bin/env python3
+"""Valid tokens/s of the padding-free GPT-3 12-layer stack on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl energon|reference]
+
+One step = one energon_stack_forward call over one batch: offsets, remove,
+12 GPT-3 layers (hidden 12288, 96 heads, FFN 49152, fp16) on the valid tokens,
+rebuild.  Default workload: batch 32, pad_len 256, every length 128 (the
+EnergonAI README's "Scaling Ability" setting: sequence length half the padding
+length).  The inputs exceed L2 (43.5 GB of weights stream through every step).
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs its own replica of the
+workload (sequences are independent, the path has no exchange step), weak
+scaling, no collective inside the timed region.  Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle (the only reference there is) on a
+bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "valid tokens/sec, GPT-3 layer stack fp16 varlen on 1 B200; % of tensor/HBM roofline"
+UNIT = "tokens/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["energon", "reference"], default="energon")
+    ap.add_argument("--workload", default="gpt3_stack_half_pad")
+    ap.add_argument("--cpu-tokens", type=int, default=0,
+                    help="tokens of the oracle's CPU sample (0: sized to about 15 s)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-padded", action="store_true")
+    ap.add_argument("--layers", type=int, default=0, help="override the workload's layer count (profiling)")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- distributed
+
+
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = False
+
+    def init(self, backend: str):
+        import torch.distributed as dist
+        if self.world > 1:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=600))
+            self.pg = True
+
+    def barrier(self):
+        if self.pg:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max(self, v: float, device) -> float:
+        if not self.pg:
+            return v
+        import torch
+        import torch.distributed as dist
+        t = torch.tensor([v], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def done(self):
+        if self.pg:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """nvidia-smi sampled every 200 ms while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.strip().splitlines():
+            p = [x.strip() for x in line.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                sm.append(float(p[1]))
+                smax.append(float(p[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, p[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------- workload
+
+
+def load_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "tflops": d["bf16_tflops"], "tflops_sustained": d["bf16_tflops_sustained"],
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "tflops": 1590.0, "tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def config_of(wl, S: int, T: int, world: int) -> dict:
+    return {"workload": wl.name, "batch": wl.batch, "pad_len": S, "valid_tokens": T, "seq_len": S,
+            "hidden": wl.shape.hidden, "heads": wl.shape.n_heads, "ffn": wl.shape.ffn, "layers": wl.n_layers,
+            "global_batch": wl.batch * world, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": "inputs larger than L2 (43.5 GB of fp16 weights stream through every step)"}
+
+
+def cpu_cores() -> int:
+    n = os.environ.get("OMP_NUM_THREADS")
+    return int(n) if n else (len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count())
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+
+def run_reference(args, dist: Dist):
+    """The oracle (fp64, C, OpenMP on the host cores) timed on a bounded sample per step.
+
+    Step i runs the first `tokens` tokens of sequence i mod batch through every layer
+    (causal attention makes a prefix exactly the work of those tokens inside the batch).
+    Layers are visited in order for all steps at once so that each layer's weights are
+    generated once; every step's time is the sum of its own per-layer oracle calls."""
+    if dist.rank != 0:
+        return
+    from padding_free_varlen_b200 import synth
+    import oracle
+    oracle.build()
+    wl = synth.WORKLOADS[args.workload]
+    lengths, S = wl.lengths(), wl.padded_len()
+    T = int(lengths.sum())
+    x = wl.x_padded()
+    tokens = args.cpu_tokens or 2
+    n = args.warmup + args.steps
+    seqs = [i % wl.batch for i in range(n)]
+    ps = [int(min(tokens, lengths[b])) for b in seqs]
+    ys = [x[b:b + 1, :p].astype(np.float64) for b, p in zip(seqs, ps)]
+    secs = [0.0] * n
+    for l in range(wl.n_layers):
+        hw = wl.layer(l)
+        for i in range(n):
+            t0 = time.perf_counter()
+            ys[i] = oracle.layer_padded(ys[i], np.array([ps[i]], np.int32), hw, wl.shape.n_heads)
+            secs[i] += time.perf_counter() - t0
+        del hw
+    total = sum(secs[args.warmup:])
+    done = sum(ps[args.warmup:])
+    value = done / total
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(wl, S, T, 1),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+                             "sample": f"per step: the first {tokens} tokens of one sequence through all "
+                                       f"{wl.n_layers} layers (fp64 C oracle; weight generation not timed)"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- our arm
+
+
+def traffic_from_profile() -> int | None:
+    """DRAM bytes per launch of the GEMM kernel from the committed ncu summary, if the kernel
+    source has not changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "gemm_tc_traffic.json")
+    src = os.path.join(ROOT, "padding_free_varlen_b200", "csrc", "gemm_tc.cu")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    if d.get("source_sha256_16") != h:
+        return None
+    return d.get("dram_bytes_per_launch_scaled")
+
+
+def run_energon(args, dist: Dist):
+    import torch
+    from padding_free_varlen_b200 import build as cuda_build
+    from padding_free_varlen_b200 import capi, synth
+
+    if dist.rank == 0 or not os.path.exists(capi.LIB_PATH):
+        cuda_build.build()
+    dist.init("nccl")
+    dist.barrier()
+    torch.cuda.set_device(dist.local)
+    dev = torch.device("cuda", dist.local)
+    wl = synth.WORKLOADS[args.workload]
+    if args.layers > 0:
+        import dataclasses
+        wl = dataclasses.replace(wl, n_layers=args.layers)
+    lengths, S = wl.lengths(), wl.padded_len()
+    B, H, L = wl.batch, wl.shape.hidden, wl.n_layers
+    T = int(lengths.sum())
+    tdt = {synth.F16: torch.float16, synth.BF16: torch.bfloat16, synth.F32: torch.float32}[wl.dtype]
+    edt = {synth.F16: capi.ENERGON_F16, synth.BF16: capi.ENERGON_BF16, synth.F32: capi.ENERGON_F32}[wl.dtype]
+    want_cpu = dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline
+
+    # ---- inputs (pinned host copies serve the end-to-end leg)
+    x_host = torch.empty((B, S, H), dtype=tdt, pin_memory=True)
+    synth.fill_normal_ptr(x_host.data_ptr(), x_host.numel(), wl.seed, synth.TID_X, wl.dtype)
+    len_host = torch.from_numpy(lengths).pin_memory()
+    d_in = x_host.to(dev)
+    d_len = len_host.to(dev)
+    d_out = torch.empty_like(d_in)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    # ---- weights: generated on the host (seeded) one layer at a time and uploaded; rank 0
+    # generates, the other ranks receive a broadcast (setup only, outside any timed region).
+    # While a layer's host copy exists, the CPU baseline runs the oracle on its sample.
+    t0 = time.perf_counter()
+    shapes = wl.shape.weight_shapes()
+    dev_layers = []
+    cpu = None
+    if want_cpu:
+        import oracle
+        oracle.build()
+        x_np = x_host.numpy() if tdt != torch.bfloat16 else x_host.view(torch.int16).numpy().view(np.uint16)
+        cpu_y, cpu_p, cpu_s = None, 0, 0.0
+    for l in range(L):
+        hw = wl.layer(l) if dist.rank == 0 else None
+        d = {}
+        for name, shp in shapes.items():
+            t = torch.empty(shp, dtype=tdt, device=dev)
+            if hw is not None:
+                src = torch.from_numpy(hw[name])
+                t.copy_(src.view(torch.bfloat16) if tdt == torch.bfloat16 else src)
+            if dist.pg:
+                import torch.distributed as tdist
+                tdist.broadcast(t, src=0)
+            d[name] = t
+        dev_layers.append(d)
+        if want_cpu:
+            if l == 0:   # size the sample to about 15 s of oracle work over all layers
+                tokens = args.cpu_tokens
+                if tokens <= 0:
+                    t1 = time.perf_counter()
+                    oracle.layer_padded(x_np[0:1, :1].astype(np.float64), np.array([1], np.int32), hw,
+                                        wl.shape.n_heads)
+                    per_tok = (time.perf_counter() - t1) * L
+                    tokens = int(max(1, min(lengths[0], 15.0 / max(per_tok, 1e-3))))
+                cpu_p = int(min(tokens, lengths[0]))
+                cpu_y = x_np[0:1, :cpu_p].astype(np.float64)
+            t1 = time.perf_counter()
+            cpu_y = oracle.layer_padded(cpu_y, np.array([cpu_p], np.int32), hw, wl.shape.n_heads)
+            cpu_s += time.perf_counter() - t1
+        del hw
+    if want_cpu:
+        cpu = {"value": cpu_p / cpu_s, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+               "sample": f"first {cpu_p} tokens of sequence 0 through all {L} layers, fp64 C oracle "
+                         f"({cpu_s:.1f} s; weight generation not timed)"}
+    tables = [capi.make_weights(d) for d in dev_layers]
+    setup_s = time.perf_counter() - t0
+
+    cfg = capi.make_config(H, wl.shape.n_heads, wl.shape.ffn, edt, wl.ln_eps)
+    ws_bytes = capi.energon_workspace_bytes(cfg, B, S)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(remove_padding=1):
+        capi.energon_stack_forward(cfg, tables, L, d_in, d_len, B, S, remove_padding, d_out, st, ws, ws_bytes,
+                                   stream)
+
+    def timed(fn, k):
+        dist.barrier()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(k):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        dist.barrier()
+        return dist.max(a.elapsed_time(b), dev)
+
+    # ---- main timed region (launch tracing on: one event pair per kernel)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(dist.local)
+    clocks.start()
+    capi.energon_trace_start()
+    ms = timed(step, args.steps)
+    trace = capi.energon_trace_stop()
+    clk = clocks.stop()
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {int(st.item())} after the timed steps")
+    value = dist.world * T * args.steps / (ms / 1e3)
+
+    # ---- roofline of the dominant kernel (the tcgen05 GEMM, four shapes per layer)
+    peaks = load_peaks()
+    gemm_names = ("gemm_qkv", "gemm_out_proj", "gemm_ffn1", "gemm_ffn2")
+    g_launch = sum(trace.get(n, (0, 0.0))[0] for n in gemm_names)
+    g_ms = sum(trace.get(n, (0, 0.0))[1] for n in gemm_names)
+    flops_per_token_layer = 24 * H * H            # 2*(3H*H + H*H + 4H*H + 4H*H)
+    gemm_flops_per_launch = flops_per_token_layer * T / 4
+    achieved = (gemm_flops_per_launch * g_launch) / (g_ms / 1e3) / 1e12 if g_ms > 0 else None
+    per_kernel = {k: {"launches": v[0], "ms_per_step": v[1] / args.steps,
+                      "share": v[1] / max(1e-9, sum(x[1] for x in trace.values()))} for k, v in trace.items()}
+    traffic = traffic_from_profile()
+    roofline = {"bound": "tensor", "kernel": "gemm_tc (tcgen05, 4 shapes per layer)",
+                "achieved": achieved, "peak": peaks["tflops_sustained"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["tflops_sustained"] if achieved else None,
+                "peak_note": f"{peaks['source']} bf16 sustained (fp16 assumed at the bf16 rate); "
+                             f"burst {peaks['tflops']}",
+                "traffic": traffic, "algorithmic_flops_per_launch": gemm_flops_per_launch,
+                "ms_per_launch": g_ms / max(1, g_launch)}
+    # memory-bound companions measured in the same region
+    aux = {}
+    e = 2 if tdt != torch.float32 else 4
+    for name, nbytes in (("remove_padding", 2 * T * H * e), ("rebuild_padding", T * H * e + B * S * H * e)):
+        if name in trace and trace[name][1] > 0:
+            gbs = nbytes * trace[name][0] / (trace[name][1] / 1e3) / 1e9
+            aux[name] = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "algorithmic_bytes_per_launch": nbytes}
+
+    # ---- end to end through the C ABI with host buffers (H2D + stack + D2H every step)
+    e2e = None
+    if not args.no_e2e:
+        out_host = torch.empty_like(x_host, pin_memory=True)
+
+        def e2e_step():
+            d_in.copy_(x_host, non_blocking=True)
+            d_len.copy_(len_host, non_blocking=True)
+            step()
+            out_host.copy_(d_out, non_blocking=True)
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        ms_e2e = timed(e2e_step, args.steps)
+        e2e = {"value": dist.world * T * args.steps / (ms_e2e / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": x_host.numel() * x_host.element_size() + len_host.numel() * 4,
+               "d2h_bytes_per_step": out_host.numel() * out_host.element_size(),
+               "ms_per_step": ms_e2e / args.steps}
+
+    # ---- the same kernels on the fully padded batch (the work elimination removes)
+    padded = None
+    if not args.no_padded:
+        kp = max(1, min(args.steps, 3))
+        step(0)
+        ms_pad = timed(lambda: step(0), kp)
+        padded = {"value": dist.world * T * kp / (ms_pad / 1e3), "unit": UNIT, "ms_per_step": ms_pad / kp,
+                  "rows_per_step": B * S, "speedup_of_packed": (ms_pad / kp) / (ms / args.steps)}
+
+    launches = sum(v[0] for v in trace.values())
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": dist.world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f16" if tdt == torch.float16 else str(tdt).replace("torch.", ""),
+            "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights)",
+            "config": config_of(wl, S, T, dist.world), "roofline": roofline, "roofline_memory_kernels": aux,
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clk,
+            "padded_path": padded, "kernels": per_kernel, "setup_s": setup_s}
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+    del tables
+    dist.done()
+
+
+def main():
+    args = parse()
+    dist = Dist()
+    if args.impl == "reference":
+        run_reference(args, dist)
+        return
+    run_energon(args, dist)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,650 @@
+// Tensor-core GEMM for sm_100a: y = A W^T + bias (+ GELU) (+ residual).
+//
+// The QKV, output-projection and FFN contractions of the GPT-3 layer, run on
+// the packed tokens only (QbitAI article "最新大模型推理系统Energon-AI开源",
+// section "Runtime": GEMM time dominates as models grow; section "易用性": the
+// bias + GELU and bias + residual steps that follow the MLP GEMMs, fused here
+// into the epilogue instead of separate passes over HBM).
+//
+// Design (one CTA per SM, persistent):
+//   - 128 x 256 output tiles, K consumed 64 elements (128 bytes) at a time.
+//   - warp 0: TMA producer.  A [rows, K] and W [N, K] tiles land in a 4-stage
+//     shared-memory ring (128-byte swizzle), completion counted on mbarriers.
+//   - warp 1: MMA issuer.  One thread issues tcgen05.mma (kind::f16, fp32
+//     accumulate) into TMEM; tcgen05.commit frees each ring slot and, at the
+//     end of a tile, hands the accumulator to the epilogue.
+//   - warp 2: allocates / frees 512 TMEM columns = two 128 x 256 fp32
+//     accumulators, so the epilogue of tile i overlaps the MMAs of tile i+1.
+//   - warps 4-7: epilogue.  tcgen05.ld (each warp owns 32 TMEM lanes = 32 rows),
+//     bias / GELU / residual in fp32, one rounding to the 16-bit type, stores.
+//   - The number of valid rows M is read on the device (cu_seqlens[batch]);
+//     tiles past M are never scheduled, rows past M are never stored.
+//   - Tiles are rasterised in groups of `group_m` row tiles so that the A
+//     panels of a group stay in L2 while the weight panels stream past once.
+//   - Every mbarrier wait is bounded: on expiry the kernel records
+//     ENERGON_DEVICE_TIMEOUT, lets the other roles stop, waits (bounded) for
+//     its copies and MMAs in flight, frees TMEM and returns.
+#include <cudaTypedefs.h>
+
+#include <stdio.h>
+
+#include <mutex>
+#include <type_traits>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace energon {
+
+namespace {
+constexpr int TBM = 128, TBN = 256, TBK = 64, TSTAGES = 4;
+constexpr int A_STAGE = TBM * TBK * 2;  // 16 KiB
+constexpr int B_STAGE = TBN * TBK * 2;  // 32 KiB
+constexpr uint32_t TMEM_COLS = 2 * TBN;
+constexpr int TC_SMEM = TSTAGES * (A_STAGE + B_STAGE) + 1024 + 256;
+
+// CTA-pair (cta_group::2) kernel: 256 x 256 tiles, each CTA stages 128 rows of A
+// and 128 rows of W (its half of the tile's N) per 64-wide K step.
+constexpr int PBM = 256, PBN = 256, PBK = 64, PSTAGES = 6;
+constexpr int PA_STAGE = 128 * PBK * 2;  // 16 KiB
+constexpr int PB_STAGE = 128 * PBK * 2;  // 16 KiB
+constexpr int P_SMEM = PSTAGES * (PA_STAGE + PB_STAGE) + 1024 + 256;
+}  // namespace
+
+struct TcParams {
+    const void* bias;
+    const void* residual;
+    void* out;
+    const int32_t* d_rows;
+    int32_t* status;
+    int M_cap, N, K, group_m, gelu_tanh;
+    uint64_t timeout_ns;
+};
+
+__device__ __forceinline__ void tile_mn(int t, int num_m, int num_n, int group_m, int& m, int& n) {
+    const int per_group = group_m * num_n;
+    const int g = t / per_group;
+    const int r = t - g * per_group;
+    const int first_m = g * group_m;
+    const int gm = min(group_m, num_m - first_m);
+    n = r / gm;
+    m = first_m + (r - n * gm);
+}
+
+// Lane 0 waits, the warp learns the outcome.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const volatile int* abort_flag,
+                                          uint64_t timeout_ns) {
+    bool ok = true;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait_bounded(bar, parity, abort_flag, timeout_ns);
+    return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
+template <typename T, int EPI>
+__device__ __forceinline__ void epilogue_store32(const uint32_t* acc, const TcParams& p, int row, int col0) {
+    float v[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(acc[j]);
+    if (p.bias != nullptr) {
+        const uint4* bp = reinterpret_cast<const uint4*>(static_cast<const T*>(p.bias) + col0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint4 w = __ldg(bp + q);
+            const uint32_t* ww = reinterpret_cast<const uint32_t*>(&w);
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                const float2 f = unpack2<T>(ww[h]);
+                v[q * 8 + 2 * h] += f.x;
+                v[q * 8 + 2 * h + 1] += f.y;
+            }
+        }
+    }
+    if (EPI == EPI_BIAS_GELU) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = gelu_f(v[j], p.gelu_tanh != 0);
+    }
+    const int64_t off = (int64_t)row * p.N + col0;
+    if (EPI == EPI_BIAS_RESIDUAL) {
+        const uint4* rp = reinterpret_cast<const uint4*>(static_cast<const T*>(p.residual) + off);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint4 w = rp[q];
+            const uint32_t* ww = reinterpret_cast<const uint32_t*>(&w);
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                const float2 f = unpack2<T>(ww[h]);
+                v[q * 8 + 2 * h] += f.x;
+                v[q * 8 + 2 * h + 1] += f.y;
+            }
+        }
+    }
+    uint4* op = reinterpret_cast<uint4*>(static_cast<T*>(p.out) + off);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        uint4 o;
+        o.x = pack2<T>(v[q * 8 + 0], v[q * 8 + 1]);
+        o.y = pack2<T>(v[q * 8 + 2], v[q * 8 + 3]);
+        o.z = pack2<T>(v[q * 8 + 4], v[q * 8 + 5]);
+        o.w = pack2<T>(v[q * 8 + 6], v[q * 8 + 7]);
+        op[q] = o;
+    }
+}
+
+template <typename T, int EPI>
+__global__ void __launch_bounds__(256, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
+                                                         const __grid_constant__ CUtensorMap tmB, const TcParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = base;
+    uint8_t* sB = base + TSTAGES * A_STAGE;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sB + TSTAGES * B_STAGE);
+    uint64_t* empty = full + TSTAGES;
+    uint64_t* tfull = empty + TSTAGES;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* drain = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (status_bad(p.status)) return;
+    const int M = min(*p.d_rows, p.M_cap);
+    if (M <= 0) return;
+    const int num_m = (M + TBM - 1) / TBM, num_n = (p.N + TBN - 1) / TBN;
+    const int total = num_m * num_n;
+    if ((int)blockIdx.x >= total) return;
+    const int num_kb = (p.K + TBK - 1) / TBK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < TSTAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], 4);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 2) {
+        tmem_alloc(tmem_slot, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- TMA producer
+        int stage = 0;
+        uint32_t phase = 0, pend_mask = 0, pend_par = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            int m, n;
+            tile_mn(t, num_m, num_n, p.group_m, m, n);
+            for (int kb = 0; kb < num_kb; ++kb) {
+                if (!warp_wait(&empty[stage], phase ^ 1u, abort_flag, p.timeout_ns)) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&full[stage], A_STAGE + B_STAGE);
+                    tma_load_2d(sA + stage * A_STAGE, &tmA, &full[stage], kb * TBK, m * TBM);
+                    tma_load_2d(sB + stage * B_STAGE, &tmB, &full[stage], kb * TBK, n * TBN);
+                }
+                pend_mask |= 1u << stage;
+                pend_par = (pend_par & ~(1u << stage)) | (phase << stage);
+                if (++stage == TSTAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        if (!ok && lane == 0) {
+            *abort_flag = 1;
+            status_or(p.status, ENERGON_DEVICE_TIMEOUT);
+            // Let every copy already issued land before the block releases its shared memory.
+            for (int s = 0; s < TSTAGES; ++s)
+                if (pend_mask & (1u << s)) mbar_wait_bounded(&full[s], (pend_par >> s) & 1u, nullptr, p.timeout_ns);
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer
+        constexpr uint32_t fmt = sizeof(T) == 2 && !std::is_same<T, __half>::value ? 1u : 0u;
+        constexpr uint32_t idesc = idesc_f16(fmt, TBM, TBN);
+        int stage = 0, local = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++local) {
+            const int acc = local & 1;
+            if (!warp_wait(&tempty[acc], ((local >> 1) & 1) ^ 1, abort_flag, p.timeout_ns)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t d_tmem = tmem + (uint32_t)(acc * TBN);
+            for (int kb = 0; kb < num_kb; ++kb) {
+                if (!warp_wait(&full[stage], phase, abort_flag, p.timeout_ns)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint64_t a0 = smem_desc_k128(smem_u32(sA + stage * A_STAGE));
+                    const uint64_t b0 = smem_desc_k128(smem_u32(sB + stage * B_STAGE));
+#pragma unroll
+                    for (int k = 0; k < TBK / 16; ++k)  // 16 elements = 32 bytes = 2 descriptor units
+                        umma_f16(d_tmem, a0 + 2 * k, b0 + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+                    umma_commit(&empty[stage]);
+                }
+                __syncwarp();
+                if (++stage == TSTAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (!ok) break;
+            if (lane == 0) umma_commit(&tfull[acc]);
+            __syncwarp();
+        }
+        if (!ok && lane == 0) {
+            *abort_flag = 1;
+            status_or(p.status, ENERGON_DEVICE_TIMEOUT);
+            umma_commit(drain);  // completes once every MMA issued so far has finished
+            mbar_wait_bounded(drain, 0, nullptr, p.timeout_ns);
+        }
+    } else if (warp >= 4) {
+        // ---------------------------------------------------------------- epilogue
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        int local = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total; t += gridDim.x, ++local) {
+            const int acc = local & 1;
+            if (!warp_wait(&tfull[acc], (local >> 1) & 1, abort_flag, p.timeout_ns)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            int m, n;
+            tile_mn(t, num_m, num_n, p.group_m, m, n);
+            const int row = m * TBM + q * 32 + lane;
+            const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * TBN);
+#pragma unroll 1
+            for (int c = 0; c < TBN; c += 32) {
+                uint32_t r[32];
+                tmem_ld_x16(tbase + c, r);
+                tmem_ld_x16(tbase + c + 16, r + 16);
+                tmem_wait_ld();
+                const int col0 = n * TBN + c;
+                if (row < M && col0 < p.N) epilogue_store32<T, EPI>(r, p, row, col0);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[acc]);
+        }
+        if (!ok && lane == 0) {
+            *abort_flag = 1;
+            status_or(p.status, ENERGON_DEVICE_TIMEOUT);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 2) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+// Spin for about `ns` nanoseconds (used only on the abort path to let copies land).
+__device__ __forceinline__ void spin_ns(uint64_t ns) {
+    const uint64_t t0 = global_ns();
+    for (uint32_t it = 0; it < (1u << 26) && global_ns() - t0 < ns; ++it) {
+    }
+}
+
+// The CTA-pair variant.  Both CTAs of a 2-CTA cluster load their halves of A
+// (by rows) and W (by the tile's columns) into their own shared memory; the
+// completion of all four copies is counted on the leader CTA's `full` barrier.
+// The leader's MMA thread issues tcgen05.mma.cta_group::2 over both CTAs'
+// shared memory; each CTA receives its 128 accumulator rows in its own TMEM.
+// Commits multicast to both CTAs (ring slots and accumulator hand-off); the
+// peer's epilogue hands accumulators back by arriving on the leader's barrier.
+template <typename T, int EPI>
+__global__ void __launch_bounds__(256, 1) gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA,
+                                                          const __grid_constant__ CUtensorMap tmB, const TcParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = base;
+    uint8_t* sB = base + PSTAGES * PA_STAGE;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sB + PSTAGES * PB_STAGE);
+    uint64_t* empty = full + PSTAGES;
+    uint64_t* tfull = empty + PSTAGES;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* drain = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    // Every early exit below is taken by both CTAs of the pair or by neither.
+    if (status_bad(p.status)) return;
+    const int M = min(*p.d_rows, p.M_cap);
+    if (M <= 0) return;
+    const int num_m = (M + PBM - 1) / PBM, num_n = (p.N + PBN - 1) / PBN;
+    const int total = num_m * num_n;
+    if (pair >= total) return;
+    const int num_kb = (p.K + PBK - 1) / PBK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < PSTAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], 8);  // 4 epilogue warps in each CTA of the pair
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 2) {
+        tmem_alloc_pair(tmem_slot, TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync();  // barriers of both CTAs initialised, TMEM of both allocated
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- TMA producer (both CTAs)
+        int stage = 0;
+        uint32_t phase = 0, pend_mask = 0, pend_par = 0;
+        bool ok = true;
+        for (int t = pair; t < total && ok; t += npairs) {
+            int m, n;
+            tile_mn(t, num_m, num_n, p.group_m, m, n);
+            for (int kb = 0; kb < num_kb; ++kb) {
+                if (!warp_wait(&empty[stage], phase ^ 1u, abort_flag, p.timeout_ns)) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) {
+                    const uint32_t bar0 = mapa_shared(smem_u32(&full[stage]), 0);
+                    if (leader) mbar_arrive_expect_tx(&full[stage], 2 * (PA_STAGE + PB_STAGE));
+                    tma_load_2d_pair(sA + stage * PA_STAGE, &tmA, bar0, kb * PBK, m * PBM + (int)rank * 128);
+                    tma_load_2d_pair(sB + stage * PB_STAGE, &tmB, bar0, kb * PBK, n * PBN + (int)rank * 128);
+                }
+                pend_mask |= 1u << stage;
+                pend_par = (pend_par & ~(1u << stage)) | (phase << stage);
+                if (++stage == PSTAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        if (!ok && lane == 0) {
+            *abort_flag = 1;
+            status_or(p.status, ENERGON_DEVICE_TIMEOUT);
+            if (leader) {
+                for (int s = 0; s < PSTAGES; ++s)
+                    if (pend_mask & (1u << s))
+                        mbar_wait_bounded(&full[s], (pend_par >> s) & 1u, nullptr, p.timeout_ns);
+            } else {
+                // The peer's copies report to the leader's barriers; give them time to land.
+                spin_ns(p.timeout_ns < 1000000ull ? p.timeout_ns : 1000000ull);
+            }
+        }
+    } else if (warp == 1 && leader) {
+        // ---------------------------------------------------------------- MMA issuer (leader CTA)
+        constexpr uint32_t fmt = sizeof(T) == 2 && !std::is_same<T, __half>::value ? 1u : 0u;
+        constexpr uint32_t idesc = idesc_f16(fmt, PBM, PBN);
+        int stage = 0, local = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int t = pair; t < total && ok; t += npairs, ++local) {
+            const int acc = local & 1;
+            if (!warp_wait(&tempty[acc], ((local >> 1) & 1) ^ 1, abort_flag, p.timeout_ns)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t d_tmem = tmem + (uint32_t)(acc * PBN);
+            for (int kb = 0; kb < num_kb; ++kb) {
+                if (!warp_wait(&full[stage], phase, abort_flag, p.timeout_ns)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint64_t a0 = smem_desc_k128(smem_u32(sA + stage * PA_STAGE));
+                    const uint64_t b0 = smem_desc_k128(smem_u32(sB + stage * PB_STAGE));
+#pragma unroll
+                    for (int k = 0; k < PBK / 16; ++k)
+                        umma_f16_pair(d_tmem, a0 + 2 * k, b0 + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+                    umma_commit_pair(&empty[stage], 0x3);
+                }
+                __syncwarp();
+                if (++stage == PSTAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (!ok) break;
+            if (lane == 0) umma_commit_pair(&tfull[acc], 0x3);
+            __syncwarp();
+        }
+        if (!ok && lane == 0) {
+            *abort_flag = 1;
+            status_or(p.status, ENERGON_DEVICE_TIMEOUT);
+            umma_commit_pair(drain, 0x1);
+            mbar_wait_bounded(drain, 0, nullptr, p.timeout_ns);
+        }
+    } else if (warp >= 4) {
+        // ---------------------------------------------------------------- epilogue (both CTAs)
+        const int q = warp & 3;
+        int local = 0;
+        bool ok = true;
+        for (int t = pair; t < total; t += npairs, ++local) {
+            const int acc = local & 1;
+            if (!warp_wait(&tfull[acc], (local >> 1) & 1, abort_flag, p.timeout_ns)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            int m, n;
+            tile_mn(t, num_m, num_n, p.group_m, m, n);
+            const int row = m * PBM + (int)rank * 128 + q * 32 + lane;
+            const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * PBN);
+#pragma unroll 1
+            for (int c = 0; c < PBN; c += 32) {
+                uint32_t r[32];
+                tmem_ld_x16(tbase + c, r);
+                tmem_ld_x16(tbase + c + 16, r + 16);
+                tmem_wait_ld();
+                const int col0 = n * PBN + c;
+                if (row < M && col0 < p.N) epilogue_store32<T, EPI>(r, p, row, col0);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
+        }
+        if (!ok && lane == 0) {
+            *abort_flag = 1;
+            status_or(p.status, ENERGON_DEVICE_TIMEOUT);
+        }
+    }
+    tc_fence_before();
+    cluster_sync();  // neither CTA leaves while its pair may still read or signal its shared memory
+    tc_fence_after();
+    if (warp == 2) tmem_dealloc_pair(tmem, TMEM_COLS);
+}
+
+// ------------------------------------------------------------------ host side
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2-D K-major tensor [rows, K] of 16-bit elements, box 64 x box_rows, 128-byte swizzle.
+static CUresult make_tmap(CUtensorMap* m, int dtype, const void* ptr, int64_t K, int64_t rows, uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return CUDA_ERROR_NOT_FOUND;
+    const CUtensorMapDataType dt =
+        dtype == ENERGON_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    cuuint32_t box[2] = {(cuuint32_t)TBK, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+bool gemm_tc_supported(const GemmArgs& a) {
+    if (a.dtype != ENERGON_F16 && a.dtype != ENERGON_BF16) return false;
+    if (a.K < TBK || a.K % TBK != 0 || a.N < TBN || a.N % TBN != 0) return false;
+    if (a.M_cap <= 0 || a.A_rows < PBM || a.A_rows % PBM != 0 || a.A_rows < a.M_cap) return false;
+    const uintptr_t al = (uintptr_t)a.A | (uintptr_t)a.W | (uintptr_t)a.out | (uintptr_t)a.bias |
+                         (uintptr_t)(a.epilogue == EPI_BIAS_RESIDUAL ? a.residual : nullptr);
+    if (al % 16 != 0) return false;
+    if (a.epilogue == EPI_BIAS_RESIDUAL && a.residual == nullptr) return false;
+    return encode_fn() != nullptr;
+}
+
+template <typename T, int EPI>
+static cudaError_t tc_launch(const CUtensorMap& ta, const CUtensorMap& tb, const TcParams& p, int grid,
+                             cudaStream_t st) {
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<T, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             TC_SMEM);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    gemm_tc_kernel<T, EPI><<<grid, 256, TC_SMEM, st>>>(ta, tb, p);
+    return cudaGetLastError();
+}
+
+template <typename T, int EPI>
+static cudaError_t tc2_launch(const CUtensorMap& ta, const CUtensorMap& tb, const TcParams& p, int pairs,
+                              cudaStream_t st) {
+    static int max_pairs = -1;
+    if (max_pairs < 0) {
+        cudaError_t e = cudaFuncSetAttribute(gemm_tc2_kernel<T, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             P_SMEM);
+        if (e != cudaSuccess) return e;
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3(2 * (device_sm_count() / 2));
+        cfg.blockDim = dim3(256);
+        cfg.dynamicSmemBytes = P_SMEM;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int clusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&clusters, gemm_tc2_kernel<T, EPI>, &cfg) != cudaSuccess || clusters < 1)
+            clusters = device_sm_count() / 2;
+        (void)cudaGetLastError();
+        max_pairs = clusters;
+    }
+    if (pairs > max_pairs) pairs = max_pairs;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * pairs);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = P_SMEM;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<T, EPI>, ta, tb, p);
+}
+
+// Single-CTA tiles for a GEMM whose rows fit in one 128-row tile (the skinny,
+// weight-streaming case): more CTAs stream weights than with 256-row pair tiles.
+static bool use_single_cta(const GemmArgs& a) { return a.M_cap <= TBM; }
+
+cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st, char* err, size_t errlen) {
+    const bool single = use_single_cta(a);
+    CUtensorMap ta, tb;
+    CUresult r1 = make_tmap(&ta, a.dtype, a.A, a.K, a.A_rows, single ? TBM : 128);
+    CUresult r2 = make_tmap(&tb, a.dtype, a.W, a.K, a.N, single ? TBN : 128);
+    if (r1 != CUDA_SUCCESS || r2 != CUDA_SUCCESS) {
+        if (err) snprintf(err, errlen, "cuTensorMapEncodeTiled failed (A: %d, W: %d)", (int)r1, (int)r2);
+        return cudaErrorInvalidValue;
+    }
+    TcParams p;
+    p.bias = a.bias;
+    p.residual = a.residual;
+    p.out = a.out;
+    p.d_rows = a.d_rows;
+    p.status = a.status;
+    p.M_cap = a.M_cap;
+    p.N = a.N;
+    p.K = a.K;
+    p.gelu_tanh = a.gelu_tanh;
+    p.timeout_ns = a.timeout_ns;
+    const bool bf = a.dtype == ENERGON_BF16;
+    if (!single) {
+        const int num_m_cap = (a.M_cap + PBM - 1) / PBM, num_n = a.N / PBN;
+        // Raster groups of 8 row tiles (2048 rows): a wave of ~74 pair tiles covers about
+        // 8 x 9 tiles, so each A and W panel is fetched into L2 about once per wave.
+        p.group_m = num_m_cap < 8 ? num_m_cap : 8;
+        const int64_t tiles_cap = (int64_t)num_m_cap * num_n;
+        const int pairs = (int)(tiles_cap < device_sm_count() / 2 ? tiles_cap : device_sm_count() / 2);
+        switch (a.epilogue) {
+        case EPI_BIAS:
+            return bf ? tc2_launch<__nv_bfloat16, EPI_BIAS>(ta, tb, p, pairs, st)
+                      : tc2_launch<__half, EPI_BIAS>(ta, tb, p, pairs, st);
+        case EPI_BIAS_GELU:
+            return bf ? tc2_launch<__nv_bfloat16, EPI_BIAS_GELU>(ta, tb, p, pairs, st)
+                      : tc2_launch<__half, EPI_BIAS_GELU>(ta, tb, p, pairs, st);
+        default:
+            return bf ? tc2_launch<__nv_bfloat16, EPI_BIAS_RESIDUAL>(ta, tb, p, pairs, st)
+                      : tc2_launch<__half, EPI_BIAS_RESIDUAL>(ta, tb, p, pairs, st);
+        }
+    }
+    const int num_m_cap = (a.M_cap + TBM - 1) / TBM, num_n = a.N / TBN;
+    // Rows of A kept hot per raster group: about 48 MiB of the 126 MB L2.
+    int gm = (int)((48ll << 20) / ((int64_t)TBM * a.K * 2));
+    p.group_m = gm < 1 ? 1 : (gm > num_m_cap ? num_m_cap : gm);
+    const int64_t tiles_cap = (int64_t)num_m_cap * num_n;
+    const int grid = (int)(tiles_cap < device_sm_count() ? tiles_cap : device_sm_count());
+    switch (a.epilogue) {
+    case EPI_BIAS:
+        return bf ? tc_launch<__nv_bfloat16, EPI_BIAS>(ta, tb, p, grid, st)
+                  : tc_launch<__half, EPI_BIAS>(ta, tb, p, grid, st);
+    case EPI_BIAS_GELU:
+        return bf ? tc_launch<__nv_bfloat16, EPI_BIAS_GELU>(ta, tb, p, grid, st)
+                  : tc_launch<__half, EPI_BIAS_GELU>(ta, tb, p, grid, st);
+    default:
+        return bf ? tc_launch<__nv_bfloat16, EPI_BIAS_RESIDUAL>(ta, tb, p, grid, st)
+                  : tc_launch<__half, EPI_BIAS_RESIDUAL>(ta, tb, p, grid, st);
+    }
+}
+
+}  // namespace energon

@@ -1,0 +1,61 @@
+// Internal launchers shared by the C-ABI layer (capi.cu) and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace energon {
+
+// Offsets: cu[b+1] = cu[b] + lengths[b]; validates lengths into *status (SET).
+cudaError_t launch_offsets(const int32_t* lengths, int batch, int pad_len, int32_t* cu, int32_t* status,
+                           cudaStream_t st);
+// cu_pad[b] = b * pad_len for b in [0, batch] (the padded path's row starts).
+cudaError_t launch_padded_starts(int batch, int pad_len, int32_t* cu_pad, const int32_t* status, cudaStream_t st);
+
+// transpose_padding_remove: packed[cu[b] + s] = padded[b, s] for s < cu[b+1] - cu[b].
+cudaError_t launch_remove(const void* padded, const int32_t* cu, int batch, int pad_len, int64_t row_bytes,
+                          void* packed, int64_t packed_rows_cap, const int32_t* status, cudaStream_t st);
+// transpose_padding_rebuild: padded[b, s] = s < len_b ? packed[starts[b] + s] : 0,
+// len_b = lens_cu[b+1] - lens_cu[b].  Writes every padded row.
+cudaError_t launch_rebuild(const void* packed, const int32_t* starts, const int32_t* lens_cu, int batch,
+                           int pad_len, int64_t row_bytes, int64_t packed_rows_cap, void* padded, cudaStream_t st);
+
+// LayerNorm over rows [0, min(*d_rows, rows_cap)) of x [rows_cap, H] -> y.
+cudaError_t launch_layernorm(int dtype, const void* x, const void* g, const void* b, void* y, const int32_t* d_rows,
+                             int rows_cap, int H, float eps, const int32_t* status, cudaStream_t st);
+
+// Epilogue variants of the GEMM y = A W^T + bias (+ GELU) (+ residual).
+enum Epilogue { EPI_BIAS = 0, EPI_BIAS_GELU = 1, EPI_BIAS_RESIDUAL = 2 };
+
+struct GemmArgs {
+    int dtype;                 // energon_dtype
+    const void* A;             // [M_cap, K]
+    const void* W;             // [N, K]
+    const void* bias;          // [N] or null
+    const void* residual;      // [M_cap, N] or null (EPI_BIAS_RESIDUAL)
+    void* out;                 // [M_cap, N]
+    const int32_t* d_rows;     // device: valid rows M (<= M_cap)
+    int M_cap, N, K;
+    int A_rows;                // rows allocated in A (>= M_cap; a multiple of 128 for the tensor-core path)
+    int epilogue;
+    int gelu_tanh;
+    int32_t* status;
+    uint64_t timeout_ns;
+};
+
+// True when the tcgen05 path can run this GEMM (16-bit types, alignment, tile multiples).
+bool gemm_tc_supported(const GemmArgs& a);
+cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st, char* err, size_t errlen);
+cudaError_t launch_gemm_simt(const GemmArgs& a, cudaStream_t st);
+
+// Causal attention within each sequence: qkv [rows, 3H] -> o [rows, H].
+cudaError_t launch_attention(int dtype, const void* qkv, void* o, const int32_t* cu, int batch, int max_len, int H,
+                             int n_heads, const int32_t* status, cudaStream_t st);
+
+// Self-test kernel of the bounded wait.
+cudaError_t launch_wait_selftest(int32_t* status, uint64_t timeout_ns, cudaStream_t st);
+
+int device_sm_count();
+
+}  // namespace energon

@@ -1,0 +1,163 @@
+// LayerNorm of the pre-LN GPT layer: y = (x - mean) / sqrt(var + eps) * g + b,
+// biased variance, statistics in fp32, output rounded to the storage type.
+// (The normalisation of the bias + residual + LayerNorm step in the QbitAI
+// article's FasterTransformer excerpt, section "易用性", placed before each
+// sub-layer as in GPT-2/3.)
+//
+// One thread block per row (grid-stride over the device-side row count).  For
+// 16-bit rows of up to 16384 elements each thread keeps its slice in registers
+// as 16-byte vectors, so the row is read from HBM once and written once.
+#include "common.cuh"
+#include "internal.h"
+
+namespace energon {
+
+// Sum over the block; every thread gets the result.  `red` holds 32 floats.
+__device__ __forceinline__ float block_sum(float v, float* red) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    __syncthreads();  // red may still be read from a previous call
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    float t = lane < nw ? red[lane] : 0.0f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    return t;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) ln_generic_kernel(const T* __restrict__ x, const T* __restrict__ g,
+                                                         const T* __restrict__ bb, T* __restrict__ y,
+                                                         const int32_t* d_rows, int rows_cap, int H, float eps,
+                                                         const int32_t* status) {
+    __shared__ float red[32];
+    if (status_bad(status)) return;
+    const int rows = min(*d_rows, rows_cap);
+    for (int r = blockIdx.x; r < rows; r += gridDim.x) {
+        const T* xr = x + (int64_t)r * H;
+        float s = 0.0f;
+        for (int k = threadIdx.x; k < H; k += blockDim.x) s += to_f(xr[k]);
+        const float mean = block_sum(s, red) / H;
+        float q = 0.0f;
+        for (int k = threadIdx.x; k < H; k += blockDim.x) {
+            float d = to_f(xr[k]) - mean;
+            q += d * d;
+        }
+        const float var = block_sum(q, red) / H;
+        const float inv = 1.0f / sqrtf(var + eps);
+        T* yr = y + (int64_t)r * H;
+        for (int k = threadIdx.x; k < H; k += blockDim.x)
+            yr[k] = from_f<T>((to_f(xr[k]) - mean) * inv * to_f(g[k]) + to_f(bb[k]));
+    }
+}
+
+// 16-bit types, H % 8 == 0, H / 8 <= 256 * VPT, 16-byte aligned pointers.
+template <typename T, int VPT>
+__global__ void __launch_bounds__(256) ln_vec_kernel(const T* __restrict__ x, const T* __restrict__ g,
+                                                     const T* __restrict__ bb, T* __restrict__ y,
+                                                     const int32_t* d_rows, int rows_cap, int H, float eps,
+                                                     const int32_t* status) {
+    __shared__ float red[32];
+    if (status_bad(status)) return;
+    const int rows = min(*d_rows, rows_cap);
+    const int nvec = H / 8;
+    for (int r = blockIdx.x; r < rows; r += gridDim.x) {
+        const uint4* xr = reinterpret_cast<const uint4*>(x + (int64_t)r * H);
+        uint4 v[VPT];
+        float s = 0.0f;
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            const int idx = i * blockDim.x + threadIdx.x;
+            if (idx < nvec) {
+                v[i] = xr[idx];
+                const uint32_t* w = reinterpret_cast<const uint32_t*>(&v[i]);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    float2 f = unpack2<T>(w[j]);
+                    s += f.x + f.y;
+                }
+            }
+        }
+        const float mean = block_sum(s, red) / H;
+        float q = 0.0f;
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            const int idx = i * blockDim.x + threadIdx.x;
+            if (idx < nvec) {
+                const uint32_t* w = reinterpret_cast<const uint32_t*>(&v[i]);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    float2 f = unpack2<T>(w[j]);
+                    q += (f.x - mean) * (f.x - mean) + (f.y - mean) * (f.y - mean);
+                }
+            }
+        }
+        const float var = block_sum(q, red) / H;
+        const float inv = 1.0f / sqrtf(var + eps);
+        uint4* yr = reinterpret_cast<uint4*>(y + (int64_t)r * H);
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            const int idx = i * blockDim.x + threadIdx.x;
+            if (idx < nvec) {
+                const uint4 gv = __ldg(reinterpret_cast<const uint4*>(g) + idx);
+                const uint4 bv = __ldg(reinterpret_cast<const uint4*>(bb) + idx);
+                const uint32_t* w = reinterpret_cast<const uint32_t*>(&v[i]);
+                const uint32_t* gw = reinterpret_cast<const uint32_t*>(&gv);
+                const uint32_t* bw = reinterpret_cast<const uint32_t*>(&bv);
+                uint4 o;
+                uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    float2 f = unpack2<T>(w[j]), gf = unpack2<T>(gw[j]), bf = unpack2<T>(bw[j]);
+                    ow[j] = pack2<T>((f.x - mean) * inv * gf.x + bf.x, (f.y - mean) * inv * gf.y + bf.y);
+                }
+                yr[idx] = o;
+            }
+        }
+    }
+}
+
+template <typename T>
+static cudaError_t ln_dispatch(const void* x, const void* g, const void* b, void* y, const int32_t* d_rows,
+                               int rows_cap, int H, float eps, const int32_t* status, cudaStream_t st) {
+    const int grid = rows_cap < 8 * device_sm_count() ? (rows_cap > 0 ? rows_cap : 1) : 8 * device_sm_count();
+    const T *xp = (const T*)x, *gp = (const T*)g, *bp = (const T*)b;
+    T* yp = (T*)y;
+    const uintptr_t al = (uintptr_t)x | (uintptr_t)g | (uintptr_t)b | (uintptr_t)y;
+    const int nvec = H / 8;
+    const int vpt = (nvec + 255) / 256;
+    if (sizeof(T) == 2 && H % 8 == 0 && al % 16 == 0 && vpt >= 1 && vpt <= 8) {
+        switch (vpt) {
+#define LN_CASE(V) \
+    case V: ln_vec_kernel<T, V><<<grid, 256, 0, st>>>(xp, gp, bp, yp, d_rows, rows_cap, H, eps, status); break;
+            LN_CASE(1) LN_CASE(2) LN_CASE(3) LN_CASE(4) LN_CASE(5) LN_CASE(6) LN_CASE(7) LN_CASE(8)
+#undef LN_CASE
+        }
+    } else {
+        ln_generic_kernel<T><<<grid, 256, 0, st>>>(xp, gp, bp, yp, d_rows, rows_cap, H, eps, status);
+    }
+    return cudaGetLastError();
+}
+
+// The vector kernel only exists for 16-bit types; fp32 always takes the generic one.
+template <>
+cudaError_t ln_dispatch<float>(const void* x, const void* g, const void* b, void* y, const int32_t* d_rows,
+                               int rows_cap, int H, float eps, const int32_t* status, cudaStream_t st) {
+    const int grid = rows_cap < 8 * device_sm_count() ? (rows_cap > 0 ? rows_cap : 1) : 8 * device_sm_count();
+    ln_generic_kernel<float><<<grid, 256, 0, st>>>((const float*)x, (const float*)g, (const float*)b, (float*)y,
+                                                   d_rows, rows_cap, H, eps, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_layernorm(int dtype, const void* x, const void* g, const void* b, void* y, const int32_t* d_rows,
+                             int rows_cap, int H, float eps, const int32_t* status, cudaStream_t st) {
+    switch (dtype) {
+    case ENERGON_F32: return ln_dispatch<float>(x, g, b, y, d_rows, rows_cap, H, eps, status, st);
+    case ENERGON_F16: return ln_dispatch<__half>(x, g, b, y, d_rows, rows_cap, H, eps, status, st);
+    case ENERGON_BF16: return ln_dispatch<__nv_bfloat16>(x, g, b, y, d_rows, rows_cap, H, eps, status, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace energon

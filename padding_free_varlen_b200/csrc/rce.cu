@@ -1,0 +1,239 @@
+// Offsets, transpose_padding_remove and transpose_padding_rebuild.
+//
+// QbitAI article "最新大模型推理系统Energon-AI开源", section "Runtime": the
+// two operators pack the valid tokens of a variable-length batch so that the
+// layers skip the padding, and scatter the result back afterwards.  The
+// packing is driven by the exclusive prefix sum of the per-sequence lengths.
+//
+// All three are HBM-bound (or launch-bound) byte movement: no tensor cores.
+// remove/rebuild move 16-byte vectors when the row size and both base
+// pointers allow it, one warp per row, grid-stride over rows; the grid is a
+// multiple of the SM count so every SM keeps several rows in flight.
+#include "common.cuh"
+#include "internal.h"
+
+namespace energon {
+
+int device_sm_count() {
+    static int sms = 0;
+    if (sms == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (sms <= 0) sms = 148;
+    }
+    return sms;
+}
+
+// ------------------------------------------------------------------ offsets
+
+__global__ void __launch_bounds__(1024) offsets_kernel(const int32_t* __restrict__ lengths, int batch, int pad_len,
+                                                      int32_t* __restrict__ cu, int32_t* __restrict__ status) {
+    __shared__ int32_t warp_tot[32];
+    __shared__ int32_t carry;
+    __shared__ int32_t bad;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+    if (tid == 0) {
+        carry = 0;
+        bad = 0;
+        cu[0] = 0;
+    }
+    __syncthreads();
+    for (int base = 0; base < batch; base += blockDim.x) {
+        const int b = base + tid;
+        const int32_t v = b < batch ? lengths[b] : 0;
+        if (b < batch && (v < 0 || v > pad_len)) bad = 1;
+        // inclusive scan inside the warp
+        int32_t x = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int32_t y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) warp_tot[warp] = x;
+        __syncthreads();
+        if (warp == 0) {
+            int32_t w = lane < nwarps ? warp_tot[lane] : 0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                int32_t y = __shfl_up_sync(0xffffffffu, w, o);
+                if (lane >= o) w += y;
+            }
+            warp_tot[lane] = w;  // inclusive totals of warps 0..lane
+        }
+        __syncthreads();
+        const int32_t incl = carry + (warp > 0 ? warp_tot[warp - 1] : 0) + x;
+        if (b < batch) cu[b + 1] = incl;
+        __syncthreads();
+        if (tid == blockDim.x - 1) carry = incl;
+        __syncthreads();
+    }
+    if (bad) {
+        for (int b = tid; b <= batch; b += blockDim.x) cu[b] = 0;
+    }
+    if (tid == 0) *status = bad ? ENERGON_DEVICE_BAD_LENGTH : ENERGON_DEVICE_OK;
+}
+
+cudaError_t launch_offsets(const int32_t* lengths, int batch, int pad_len, int32_t* cu, int32_t* status,
+                           cudaStream_t st) {
+    int threads = batch >= 1024 ? 1024 : ((batch + 31) / 32) * 32;
+    if (threads < 32) threads = 32;
+    offsets_kernel<<<1, threads, 0, st>>>(lengths, batch, pad_len, cu, status);
+    return cudaGetLastError();
+}
+
+__global__ void padded_starts_kernel(int batch, int pad_len, int32_t* cu_pad) {
+    for (int b = blockIdx.x * blockDim.x + threadIdx.x; b <= batch; b += gridDim.x * blockDim.x)
+        cu_pad[b] = b * pad_len;
+}
+
+cudaError_t launch_padded_starts(int batch, int pad_len, int32_t* cu_pad, const int32_t*, cudaStream_t st) {
+    int blocks = (batch + 1 + 255) / 256;
+    padded_starts_kernel<<<blocks, 256, 0, st>>>(batch, pad_len, cu_pad);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ remove / rebuild
+
+// Largest b in [0, batch) with cu[b] <= r (the sequence that owns packed row r).
+__device__ __forceinline__ int owner_of(const int32_t* __restrict__ cu, int batch, int64_t r) {
+    int lo = 0, hi = batch - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (__ldg(cu + mid) <= r) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
+template <typename V, int UNROLL>
+__device__ __forceinline__ void warp_copy_row(const V* __restrict__ src, V* __restrict__ dst, int64_t nvec, int lane) {
+    for (int64_t base = lane; base < nvec; base += 32 * UNROLL) {
+        V tmp[UNROLL];
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u) {
+            int64_t i = base + (int64_t)u * 32;
+            if (i < nvec) tmp[u] = __ldcs(src + i);
+        }
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u) {
+            int64_t i = base + (int64_t)u * 32;
+            if (i < nvec) dst[i] = tmp[u];
+        }
+    }
+}
+
+template <typename V>
+__device__ __forceinline__ void warp_zero_row(V* __restrict__ dst, int64_t nvec, int lane) {
+    V z;
+    memset(&z, 0, sizeof(V));
+    for (int64_t i = lane; i < nvec; i += 32) __stcs(dst + i, z);
+}
+
+template <typename V, int UNROLL>
+__global__ void __launch_bounds__(256) remove_kernel(const V* __restrict__ padded, const int32_t* __restrict__ cu,
+                                                     int batch, int pad_len, int64_t row_vecs, V* __restrict__ packed,
+                                                     int64_t packed_rows_cap, const int32_t* status) {
+    if (status_bad(status) || batch <= 0) return;
+    int64_t T = __ldg(cu + batch);
+    const int64_t cap = (int64_t)batch * pad_len;
+    if (T > cap) T = cap;
+    if (T > packed_rows_cap) T = packed_rows_cap;
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < T; r += warps) {
+        const int b = owner_of(cu, batch, r);
+        const int64_t s = r - __ldg(cu + b);
+        if (s < 0 || s >= pad_len) continue;  // offsets inconsistent with pad_len: skip the row
+        warp_copy_row<V, UNROLL>(padded + ((int64_t)b * pad_len + s) * row_vecs, packed + r * row_vecs, row_vecs,
+                                 lane);
+    }
+}
+
+template <typename V, int UNROLL>
+__global__ void __launch_bounds__(256) rebuild_kernel(const V* __restrict__ packed, const int32_t* __restrict__ starts,
+                                                      const int32_t* __restrict__ lens_cu, int batch, int pad_len,
+                                                      int64_t row_vecs, int64_t packed_rows_cap, V* __restrict__ padded) {
+    const int lane = threadIdx.x & 31;
+    const int64_t rows = (int64_t)batch * pad_len;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
+        const int b = (int)(r / pad_len);
+        const int s = (int)(r - (int64_t)b * pad_len);
+        const int len = __ldg(lens_cu + b + 1) - __ldg(lens_cu + b);
+        const int64_t src = (int64_t)__ldg(starts + b) + s;
+        V* dst = padded + r * row_vecs;
+        if (s < len && src >= 0 && src < packed_rows_cap)
+            warp_copy_row<V, UNROLL>(packed + src * row_vecs, dst, row_vecs, lane);
+        else
+            warp_zero_row<V>(dst, row_vecs, lane);
+    }
+}
+
+static int row_grid(int64_t rows) {
+    const int64_t per_sm = 8;  // 8 blocks of 8 warps = 64 warps per SM
+    int64_t want = (rows + 7) / 8;
+    int64_t cap = per_sm * device_sm_count();
+    if (want > cap) want = cap;
+    if (want < 1) want = 1;
+    return (int)want;
+}
+
+cudaError_t launch_remove(const void* padded, const int32_t* cu, int batch, int pad_len, int64_t row_bytes,
+                          void* packed, int64_t packed_rows_cap, const int32_t* status, cudaStream_t st) {
+    if (batch <= 0 || row_bytes == 0) return cudaSuccess;
+    const int grid = row_grid((int64_t)batch * pad_len);
+    const uintptr_t align = reinterpret_cast<uintptr_t>(padded) | reinterpret_cast<uintptr_t>(packed);
+    if (row_bytes % 16 == 0 && align % 16 == 0) {
+        remove_kernel<uint4, 4><<<grid, 256, 0, st>>>((const uint4*)padded, cu, batch, pad_len, row_bytes / 16,
+                                                      (uint4*)packed, packed_rows_cap, status);
+    } else if (row_bytes % 4 == 0 && align % 4 == 0) {
+        remove_kernel<uint32_t, 8><<<grid, 256, 0, st>>>((const uint32_t*)padded, cu, batch, pad_len, row_bytes / 4,
+                                                         (uint32_t*)packed, packed_rows_cap, status);
+    } else {
+        remove_kernel<uint8_t, 8><<<grid, 256, 0, st>>>((const uint8_t*)padded, cu, batch, pad_len, row_bytes,
+                                                        (uint8_t*)packed, packed_rows_cap, status);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_rebuild(const void* packed, const int32_t* starts, const int32_t* lens_cu, int batch, int pad_len,
+                           int64_t row_bytes, int64_t packed_rows_cap, void* padded, cudaStream_t st) {
+    if (batch <= 0 || pad_len <= 0 || row_bytes == 0) return cudaSuccess;
+    const int grid = row_grid((int64_t)batch * pad_len);
+    const uintptr_t align = reinterpret_cast<uintptr_t>(padded) | reinterpret_cast<uintptr_t>(packed);
+    if (row_bytes % 16 == 0 && align % 16 == 0) {
+        rebuild_kernel<uint4, 4><<<grid, 256, 0, st>>>((const uint4*)packed, starts, lens_cu, batch, pad_len,
+                                                       row_bytes / 16, packed_rows_cap, (uint4*)padded);
+    } else if (row_bytes % 4 == 0 && align % 4 == 0) {
+        rebuild_kernel<uint32_t, 8><<<grid, 256, 0, st>>>((const uint32_t*)packed, starts, lens_cu, batch, pad_len,
+                                                          row_bytes / 4, packed_rows_cap, (uint32_t*)padded);
+    } else {
+        rebuild_kernel<uint8_t, 8><<<grid, 256, 0, st>>>((const uint8_t*)packed, starts, lens_cu, batch, pad_len,
+                                                         row_bytes, packed_rows_cap, (uint8_t*)padded);
+    }
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ bounded-wait self-test
+
+__global__ void wait_selftest_kernel(int32_t* status, uint64_t timeout_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        // Nobody arrives on `bar`: the wait must give up by itself.
+        if (!mbar_wait_bounded(&bar, 0, nullptr, timeout_ns)) status_or(status, ENERGON_DEVICE_TIMEOUT);
+    }
+    __syncthreads();
+}
+
+cudaError_t launch_wait_selftest(int32_t* status, uint64_t timeout_ns, cudaStream_t st) {
+    wait_selftest_kernel<<<1, 32, 0, st>>>(status, timeout_ns);
+    return cudaGetLastError();
+}
+
+}  // namespace energon

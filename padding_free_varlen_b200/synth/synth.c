@@ -17,8 +17,9 @@
  * Element i of a normal tensor is mean + std * z_{i mod 2} of pair p = i / 2.
  * Uniform integers in [lo, hi] are lo + floor(u * (hi - lo + 1)).
  *
- * Storage rounding is round-to-nearest-even, done here by exact scaling and
- * nearbyint() so that it does not depend on compiler half-precision support.
+ * Storage rounding is round-to-nearest-even, done on the binary64 bit fields
+ * with integer arithmetic so that it does not depend on compiler
+ * half-precision support or on the floating-point rounding mode.
  */
 #include <math.h>
 #include <stdint.h>
@@ -45,41 +46,61 @@ static inline uint64_t draw(uint64_t base, uint64_t c) { return mix64(base + (c 
 
 static inline double to_unit(uint64_t r) { return (double)(r >> 11) * 0x1p-53; }
 
-/* x -> IEEE binary16 bits, round to nearest even. */
-static uint16_t round_f16(double x) {
-    uint16_t sign = signbit(x) ? 0x8000u : 0u;
-    double a = fabs(x);
-    if (isnan(a)) return (uint16_t)(sign | 0x7E00u);
-    if (a >= 65520.0) return (uint16_t)(sign | 0x7C00u);
-    if (a < 0x1p-14) {
-        double q = nearbyint(a * 0x1p24); /* subnormal units of 2^-24; 1024 encodes 2^-14 */
-        return (uint16_t)(sign | (uint16_t)q);
-    }
-    int e;
-    double m = frexp(a, &e); /* a = m 2^e, m in [0.5, 1) */
-    double q = nearbyint(ldexp(m, 11));
-    if (q == 2048.0) { q = 1024.0; e += 1; }
-    int E = e + 14;
-    if (E >= 31) return (uint16_t)(sign | 0x7C00u);
-    return (uint16_t)(sign | (uint16_t)(E << 10) | (uint16_t)((int)q - 1024));
+/* Round a non-negative finite significand m (53 bits, implicit bit set) right
+ * by `shift` bits, to nearest, ties to even. */
+static inline uint64_t rne_shift(uint64_t m, int shift) {
+    if (shift >= 64) return 0;
+    if (shift <= 0) return m;
+    uint64_t q = m >> shift;
+    uint64_t rem = m & ((1ULL << shift) - 1);
+    uint64_t half = 1ULL << (shift - 1);
+    if (rem > half || (rem == half && (q & 1))) ++q;
+    return q;
 }
 
-/* x -> bfloat16 bits, round to nearest even. */
-static uint16_t round_bf16(double x) {
-    uint16_t sign = signbit(x) ? 0x8000u : 0u;
-    double a = fabs(x);
-    if (isnan(a)) return (uint16_t)(sign | 0x7FC0u);
-    if (a < 0x1p-126) {
-        double q = nearbyint(a * 0x1p133); /* subnormal units of 2^-133 */
-        return (uint16_t)(sign | (uint16_t)q);
+/* x -> IEEE binary16 bits, round to nearest even, from the binary64 fields. */
+static uint16_t round_f16(double x) {
+    uint64_t b;
+    memcpy(&b, &x, 8);
+    uint16_t sign = (uint16_t)((b >> 48) & 0x8000u);
+    int e = (int)((b >> 52) & 0x7FF);
+    uint64_t frac = b & ((1ULL << 52) - 1);
+    if (e == 0x7FF) return (uint16_t)(sign | (frac ? 0x7E00u : 0x7C00u));
+    if (e == 0) return sign; /* binary64 subnormals are far below half the smallest f16 */
+    int ue = e - 1023;
+    uint64_t m = frac | (1ULL << 52);
+    if (ue >= -14) { /* normal f16 range (before rounding) */
+        uint64_t q = rne_shift(m, 42);        /* 11-bit significand, in [1024, 2048] */
+        if (q == 2048) { q = 1024; ++ue; }
+        int E = ue + 15;
+        if (E >= 31) return (uint16_t)(sign | 0x7C00u);
+        return (uint16_t)(sign | (uint16_t)(E << 10) | (uint16_t)(q - 1024));
     }
-    int e;
-    double m = frexp(a, &e);
-    double q = nearbyint(ldexp(m, 8));
-    if (q == 256.0) { q = 128.0; e += 1; }
-    int E = e + 126;
-    if (E >= 255) return (uint16_t)(sign | 0x7F80u);
-    return (uint16_t)(sign | (uint16_t)(E << 7) | (uint16_t)((int)q - 128));
+    /* subnormal f16: units of 2^-24; value = m 2^(ue-52) */
+    uint64_t q = rne_shift(m, 42 + (-14 - ue));
+    return (uint16_t)(sign | (uint16_t)q); /* q == 1024 encodes 2^-14 */
+}
+
+/* x -> bfloat16 bits, round to nearest even, from the binary64 fields. */
+static uint16_t round_bf16(double x) {
+    uint64_t b;
+    memcpy(&b, &x, 8);
+    uint16_t sign = (uint16_t)((b >> 48) & 0x8000u);
+    int e = (int)((b >> 52) & 0x7FF);
+    uint64_t frac = b & ((1ULL << 52) - 1);
+    if (e == 0x7FF) return (uint16_t)(sign | (frac ? 0x7FC0u : 0x7F80u));
+    if (e == 0) return sign;
+    int ue = e - 1023;
+    uint64_t m = frac | (1ULL << 52);
+    if (ue >= -126) {
+        uint64_t q = rne_shift(m, 45);        /* 8-bit significand, in [128, 256] */
+        if (q == 256) { q = 128; ++ue; }
+        int E = ue + 127;
+        if (E >= 255) return (uint16_t)(sign | 0x7F80u);
+        return (uint16_t)(sign | (uint16_t)(E << 7) | (uint16_t)(q - 128));
+    }
+    uint64_t q = rne_shift(m, 45 + (-126 - ue)); /* units of 2^-133 */
+    return (uint16_t)(sign | (uint16_t)q);
 }
 
 static inline void store(void* out, int dtype, int64_t i, double v) {
@@ -98,15 +119,17 @@ int synth_normal(uint64_t seed, uint64_t tensor, int64_t offset, int64_t n, doub
     if (n < 0 || offset < 0 || !out || dtype < 0 || dtype > 3) return 1;
     const uint64_t base = stream_base(seed, tensor);
     const double two_pi = 6.283185307179586476925286766559;
+    /* Pairs p cover elements 2p and 2p + 1; each pair's Box-Muller step runs once. */
+    const int64_t p0 = offset >> 1, p1 = (offset + n + 1) >> 1;
 #pragma omp parallel for schedule(static)
-    for (int64_t j = 0; j < n; ++j) {
-        int64_t i = offset + j;
-        uint64_t p = (uint64_t)(i >> 1);
-        double u0 = to_unit(draw(base, 2 * p));
-        double u1 = to_unit(draw(base, 2 * p + 1));
+    for (int64_t p = p0; p < p1; ++p) {
+        double u0 = to_unit(draw(base, 2 * (uint64_t)p));
+        double u1 = to_unit(draw(base, 2 * (uint64_t)p + 1));
         double rho = sqrt(-2.0 * log(1.0 - u0));
-        double z = (i & 1) ? rho * sin(two_pi * u1) : rho * cos(two_pi * u1);
-        store(out, dtype, j, mean + std * z);
+        double ang = two_pi * u1;
+        int64_t i0 = 2 * p - offset, i1 = i0 + 1;
+        if (i0 >= 0 && i0 < n) store(out, dtype, i0, mean + std * (rho * cos(ang)));
+        if (i1 >= 0 && i1 < n) store(out, dtype, i1, mean + std * (rho * sin(ang)));
     }
     return 0;
 }

@@ -1,0 +1,115 @@
+"""The C-ABI library without a GPU: it builds, loads, exports every declared
+symbol, and refuses bad arguments on the host before any launch."""
+import ctypes
+import glob
+import os
+import re
+import subprocess
+
+import pytest
+
+from padding_free_varlen_b200 import build as pbuild
+from padding_free_varlen_b200 import capi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    pbuild.build()
+    return capi.load()
+
+
+def declared_symbols():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        names += re.findall(r"ENERGON_API\s+[\w\s\*]+?\b(energon_\w+)\s*\(", open(h).read())
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_symbols()
+    assert len(names) >= 9
+    out = subprocess.run(["nm", "-D", "--defined-only", capi.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (energon_\w+)", out))
+    assert set(names) <= exported, set(names) - exported
+    assert set(capi.EXPORTED) == set(names)
+    for n in names:
+        assert hasattr(lib, n)
+
+
+def test_library_is_built_for_sm100a(lib):
+    out = subprocess.run(["cuobjdump", "--list-elf", capi.LIB_PATH], capture_output=True, text=True).stdout
+    assert "sm_100a" in out
+
+
+def cfg(H=256, nh=2, F=1024, dtype=capi.ENERGON_F16):
+    return capi.make_config(H, nh, F, dtype)
+
+
+def test_workspace_bytes_matches_documented_layout(lib):
+    def align(v, a):
+        return (v + a - 1) // a * a
+    for (H, nh, F, dt, e, B, S) in [(256, 2, 1024, capi.ENERGON_F16, 2, 3, 70),
+                                   (12288, 96, 49152, capi.ENERGON_F16, 2, 32, 256),
+                                   (256, 4, 1024, capi.ENERGON_F32, 4, 4, 32)]:
+        R = align(B * S, 256)
+        off = 0
+        for cols in (H, 3 * H, H, H, F, H):
+            off = align(off + R * cols * e, 1024)
+        off = align(off + (B + 1) * 4, 1024)
+        off = align(off + (B + 1) * 4, 1024)
+        assert capi.energon_workspace_bytes(cfg(H, nh, F, dt), B, S) == off
+
+
+def test_workspace_bytes_invalid_config(lib):
+    assert capi.energon_workspace_bytes(cfg(H=250), 2, 8) == 0          # head_dim 125
+    assert capi.energon_workspace_bytes(cfg(dtype=7), 2, 8) == 0
+    assert capi.energon_workspace_bytes(cfg(), 0, 8) == 0
+
+
+def test_bad_arguments_fail_before_launch(lib):
+    # Each call below is refused by the host-side checks, so no kernel is launched.
+    with pytest.raises(capi.EnergonError) as e:
+        capi.energon_rce_offsets(None, 4, 8, None, None, stream=0)
+    assert e.value.code == capi.ENERGON_ERR_INVALID_ARGUMENT
+    with pytest.raises(capi.EnergonError) as e:
+        capi.energon_rce_remove_padding(None, None, 1, 1, 1, 2, None, stream=0)
+    assert e.value.code == capi.ENERGON_ERR_INVALID_ARGUMENT
+    with pytest.raises(capi.EnergonError) as e:
+        capi.energon_rce_rebuild_padding(None, None, 1, 1, 1, 2, None, stream=0)
+    assert e.value.code == capi.ENERGON_ERR_INVALID_ARGUMENT
+    w = capi.energon_layer_weights(*([0] * 12))
+    with pytest.raises(capi.EnergonError) as e:
+        capi.energon_layer_forward(cfg(), w, 0, 0, 2, 8, 0, 0, 0, 0, stream=0)
+    assert e.value.code == capi.ENERGON_ERR_INVALID_ARGUMENT
+    assert "weight" in capi.energon_last_error()
+    with pytest.raises(capi.EnergonError) as e:
+        capi.energon_stack_forward(cfg(H=384, nh=4), [w], 1, 0, 0, 2, 8, 1, 0, 0, 0, 0, stream=0)
+    assert e.value.code == capi.ENERGON_ERR_UNSUPPORTED                     # head_dim 96
+    with pytest.raises(capi.EnergonError) as e:
+        capi.energon_stack_forward(cfg(), [w], 1, 0, 0, 0, 8, 1, 0, 0, 0, 0, stream=0)
+    assert e.value.code == capi.ENERGON_ERR_INVALID_ARGUMENT                # batch 0
+    fake = capi.energon_layer_weights(*([4096] * 12))
+    with pytest.raises(capi.EnergonError) as e:   # workspace of 0 bytes is always too small
+        capi.energon_stack_forward(cfg(), [fake], 1, 4096, 8192, 2, 8, 1, 12288, 16384, 20480, 0, stream=0)
+    assert e.value.code == capi.ENERGON_ERR_WORKSPACE_TOO_SMALL
+    with pytest.raises(capi.EnergonError) as e:
+        capi.energon_stack_forward(cfg(), [fake], 1, 4096, 8192, 2, 8, 1, 4096, 16384, 20480, 1 << 40, stream=0)
+    assert e.value.code == capi.ENERGON_ERR_INVALID_ARGUMENT                # out aliases in
+    with pytest.raises(capi.EnergonError):
+        capi.energon_selftest_bounded_wait(None, 10, stream=0)
+
+
+def test_binding_rejects_host_tensors(lib):
+    import torch
+    with pytest.raises(ValueError):
+        capi.energon_rce_offsets(torch.zeros(4, dtype=torch.int32), 4, 8, torch.zeros(5, dtype=torch.int32),
+                                 torch.zeros(1, dtype=torch.int32), stream=0)
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    monkeypatch.setattr(capi, "_lib", None)
+    monkeypatch.setattr(capi, "LIB_PATH", str(tmp_path / "absent.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        capi.load()
