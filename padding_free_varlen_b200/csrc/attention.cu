@@ -8,7 +8,8 @@
 // packed tokens only (EnergonAI README, "Scaling Ability": redundant
 // computation elimination in the GPT-3 layers).
 //
-// CUDA-core kernel: one block per (64-query tile, head, sequence), 8 warps,
+// CUDA-core kernel (fp32, head_dim 64; the 16-bit head_dim-128 case runs on the
+// tensor cores, attention_tc.cu): one block per (64-query tile, head, sequence), 8 warps,
 // each warp owning 8 queries; keys and values are staged through shared
 // memory 64 at a time and combined with an online (running-max) softmax in
 // fp32.  Key chunks beyond a query are fully masked and leave its state
@@ -151,8 +152,10 @@ static cudaError_t attn_launch(const void* qkv, void* o, const int32_t* cu, int 
 }
 
 cudaError_t launch_attention(int dtype, const void* qkv, void* o, const int32_t* cu, int batch, int max_len, int H,
-                             int n_heads, const int32_t* status, cudaStream_t st) {
+                             int n_heads, int qkv_rows, int32_t* status, uint64_t timeout_ns, cudaStream_t st) {
     if (batch <= 0 || max_len <= 0) return cudaSuccess;
+    if (attention_tc_supported(dtype, H, n_heads, qkv, o, qkv_rows))
+        return launch_attention_tc(dtype, qkv, o, cu, batch, max_len, H, n_heads, qkv_rows, status, timeout_ns, st);
     const int hd = H / n_heads;
     if (hd != 64 && hd != 128) return cudaErrorInvalidValue;
 #define ATTN_CASE(T)                                                                                     \

@@ -1,0 +1,327 @@
+// Causal self-attention on packed tokens with the 5th-generation tensor cores.
+//
+// The attention of the GPT-3 layer run on the valid tokens only (EnergonAI
+// README, "Scaling Ability": redundant computation elimination), driven by
+// cu_seqlens: sequence b owns packed rows cu[b] .. cu[b+1]-1 of the fused
+// projection qkv [rows, 3H] (columns Q | K | V, head-major inside each).  For
+// head j and position s:  o_j(s) = sum_{t <= s} softmax_t(q_j(s) . k_j(t) / sqrt(d)) v_j(t).
+//
+// One CTA = 128 queries of one (sequence, head), head_dim 128, 128 threads;
+// thread i owns query row i, which is TMEM lane i.  Per 128-key block:
+//   TMA   Q (once), K and V tiles straight from the packed qkv rows (128-byte swizzle)
+//   MMA   S = Q K^T  (tcgen05.mma kind::f16, M = N = K = 128) into TMEM columns 0..127
+//   ALU   each thread reads its S row from TMEM, applies the causal mask, keeps
+//         a running max / sum (online softmax, fp32, exp2 with the scale folded
+//         in) and writes P, rounded to the storage type, into shared memory
+//   MMA   O += P V  (V used as an MN-major operand, no transpose) into TMEM 128..255
+// Keys past the sequence are masked; their V rows are zeroed in shared memory
+// first, so stale workspace contents can never reach a valid row (0 * NaN).
+// Causality bounds the key blocks of query tile qb to 0..qb, so a query visits
+// the same blocks whether its sequence is packed or padded.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+#include <type_traits>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace energon {
+
+namespace {
+constexpr int ATQ = 128;                // queries per CTA
+constexpr int ATK = 128;                // keys per block
+constexpr int AHD = 128;                // head dim
+constexpr int ATILE = 128 * 64 * 2;     // 128 rows x 64 columns of 16-bit = 16 KiB, one swizzle block column
+constexpr int AT_SMEM = 6 * ATILE + 1024 + 128;
+constexpr uint32_t AT_TMEM_COLS = 256;  // S: 0..127, O: 128..255
+}  // namespace
+
+struct AttnTcParams {
+    const int32_t* cu;
+    void* out;
+    int32_t* status;
+    int H;
+    float scale_log2e;  // log2(e) / sqrt(head_dim)
+    uint64_t timeout_ns;
+};
+
+// Thread 0 waits (bounded); every thread learns the outcome at the same barrier.
+__device__ __forceinline__ bool block_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
+    int ok = 1;
+    if (threadIdx.x == 0) ok = mbar_wait_bounded(bar, parity, nullptr, timeout_ns) ? 1 : 0;
+    return __syncthreads_and(ok) != 0;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(128) attn_tc_kernel(const __grid_constant__ CUtensorMap tm, const AttnTcParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sQ = base;              // Q: head dims 0..63 | 64..127
+    uint8_t* sK = base + 2 * ATILE;  // K: head dims 0..63 | 64..127; then P: keys 0..63 | 64..127
+    uint8_t* sV = base + 4 * ATILE;  // V: head dims 0..63 | 64..127, one row per key
+    uint64_t* bars = reinterpret_cast<uint64_t*>(base + 6 * ATILE);
+    uint64_t* bar_q = bars;
+    uint64_t* bar_kv = bars + 1;
+    uint64_t* bar_mma = bars + 2;
+    uint64_t* drain = bars + 3;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
+
+    const int tid = threadIdx.x, warp = tid >> 5;
+    if (status_bad(p.status)) return;
+    const int b = blockIdx.z, j = blockIdx.y, q0 = blockIdx.x * ATQ;
+    const int start = p.cu[b], len = p.cu[b + 1] - start;
+    if (q0 >= len) return;
+    const int n_kb = q0 / ATK + 1;  // causal: key blocks 0 .. the diagonal one
+    const int q = q0 + tid;
+    const bool row_ok = q < len;
+
+    if (tid == 0) {
+        for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, AT_TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const uint32_t S_t = tmem + lane_base, O_t = tmem + lane_base + 128;
+
+    const int colQ = j * AHD, colK = p.H + j * AHD, colV = 2 * p.H + j * AHD;
+    bool q_pending = false, kv_pending = false;
+    uint32_t kv_parity = 0;
+    if (tid == 0) {
+        tma_prefetch_desc(&tm);
+        mbar_arrive_expect_tx(bar_q, 2 * ATILE);
+        tma_load_2d(sQ, &tm, bar_q, colQ, start + q0);
+        tma_load_2d(sQ + ATILE, &tm, bar_q, colQ + 64, start + q0);
+        mbar_arrive_expect_tx(bar_kv, 4 * ATILE);
+        tma_load_2d(sK, &tm, bar_kv, colK, start);
+        tma_load_2d(sK + ATILE, &tm, bar_kv, colK + 64, start);
+        tma_load_2d(sV, &tm, bar_kv, colV, start);
+        tma_load_2d(sV + ATILE, &tm, bar_kv, colV + 64, start);
+        q_pending = kv_pending = true;
+    }
+    constexpr uint32_t fmt = std::is_same<T, __half>::value ? 0u : 1u;
+    constexpr uint32_t idesc_s = idesc_f16(fmt, ATQ, ATK, 0);
+    constexpr uint32_t idesc_o = idesc_f16(fmt, ATQ, AHD, 1);
+
+    float m_i = -INFINITY, l_i = 0.0f;
+    uint32_t mma_phase = 0;
+    bool ok = block_wait(bar_q, 0, p.timeout_ns);
+    if (ok) q_pending = false;
+    uint32_t r[32];
+    for (int kb = 0; ok && kb < n_kb; ++kb) {
+        ok = block_wait(bar_kv, kv_parity, p.timeout_ns);
+        if (!ok) break;
+        kv_pending = false;
+        kv_parity ^= 1u;
+        const int kbase = kb * ATK;
+        if (kbase + tid >= len) {  // key row past the sequence: zero its V row
+            uint4 z = make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                reinterpret_cast<uint4*>(sV + tid * 128)[c] = z;
+                reinterpret_cast<uint4*>(sV + ATILE + tid * 128)[c] = z;
+            }
+            fence_proxy_async_smem();
+        }
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int k = 0; k < AHD / 16; ++k) {
+                const uint64_t a = smem_desc_k128(smem_u32(sQ + (k >> 2) * ATILE)) + 2 * (k & 3);
+                const uint64_t bk = smem_desc_k128(smem_u32(sK + (k >> 2) * ATILE)) + 2 * (k & 3);
+                umma_f16(tmem, a, bk, idesc_s, k > 0 ? 1u : 0u);
+            }
+            umma_commit(bar_mma);
+        }
+        ok = block_wait(bar_mma, mma_phase, p.timeout_ns);
+        mma_phase ^= 1u;
+        if (!ok) break;
+        tc_fence_after();
+
+        // ---- online softmax of this thread's row
+        const int nvalid = row_ok ? min(ATK, q - kbase + 1) : 0;  // keys kbase .. kbase+nvalid-1 are visible
+        float mx = -INFINITY;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+            tmem_ld_x32(S_t + c * 32, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+                if (c * 32 + e < nvalid) mx = fmaxf(mx, __uint_as_float(r[e]));
+        }
+        const float m_new = row_ok ? fmaxf(m_i, mx) : 0.0f;
+        const float alpha = row_ok ? exp2f((m_i - m_new) * p.scale_log2e) : 1.0f;
+        float rs = 0.0f;
+        uint8_t* sP = sK;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+            tmem_ld_x32(S_t + c * 32, r);
+            tmem_wait_ld();
+            float pv[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                pv[e] = (c * 32 + e < nvalid) ? exp2f((__uint_as_float(r[e]) - m_new) * p.scale_log2e) : 0.0f;
+                rs += pv[e];
+            }
+            // keys c*32 .. c*32+31: swizzle block c/2, 16-byte chunks (c%2)*4 .. +3 of row tid
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                uint4 w;
+                w.x = pack2<T>(pv[8 * g + 0], pv[8 * g + 1]);
+                w.y = pack2<T>(pv[8 * g + 2], pv[8 * g + 3]);
+                w.z = pack2<T>(pv[8 * g + 4], pv[8 * g + 5]);
+                w.w = pack2<T>(pv[8 * g + 6], pv[8 * g + 7]);
+                const int ch = (c & 1) * 4 + g;
+                *reinterpret_cast<uint4*>(sP + (c >> 1) * ATILE + tid * 128 + ((ch ^ (tid & 7)) << 4)) = w;
+            }
+        }
+        l_i = l_i * alpha + rs;
+        if (row_ok) m_i = m_new;
+        if (kb > 0) {  // earlier blocks were summed against a smaller max: rescale O
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                tmem_ld_x32(O_t + c * 32, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+                tmem_st_x32(O_t + c * 32, r);
+            }
+            tmem_wait_st();
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int k = 0; k < ATK / 16; ++k) {
+                const uint64_t a = smem_desc_k128(smem_u32(sP + (k >> 2) * ATILE)) + 2 * (k & 3);
+                const uint64_t bv = smem_desc_mn128(smem_u32(sV + k * 2048), ATILE, 1024);
+                umma_f16(tmem + 128, a, bv, idesc_o, (kb > 0 || k > 0) ? 1u : 0u);
+            }
+            umma_commit(bar_mma);
+        }
+        ok = block_wait(bar_mma, mma_phase, p.timeout_ns);
+        mma_phase ^= 1u;
+        if (!ok) break;
+        tc_fence_after();
+        if (kb + 1 < n_kb && tid == 0) {
+            const int y = start + (kb + 1) * ATK;
+            mbar_arrive_expect_tx(bar_kv, 4 * ATILE);
+            tma_load_2d(sK, &tm, bar_kv, colK, y);
+            tma_load_2d(sK + ATILE, &tm, bar_kv, colK + 64, y);
+            tma_load_2d(sV, &tm, bar_kv, colV, y);
+            tma_load_2d(sV + ATILE, &tm, bar_kv, colV + 64, y);
+            kv_pending = true;
+        }
+    }
+    if (ok) {
+        const float inv = row_ok ? 1.0f / l_i : 0.0f;
+        T* orow = static_cast<T*>(p.out) + (int64_t)(start + q) * p.H + j * AHD;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+            tmem_ld_x32(O_t + c * 32, r);
+            tmem_wait_ld();
+            if (row_ok) {
+                uint4* op = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    uint4 w;
+                    w.x = pack2<T>(__uint_as_float(r[8 * g + 0]) * inv, __uint_as_float(r[8 * g + 1]) * inv);
+                    w.y = pack2<T>(__uint_as_float(r[8 * g + 2]) * inv, __uint_as_float(r[8 * g + 3]) * inv);
+                    w.z = pack2<T>(__uint_as_float(r[8 * g + 4]) * inv, __uint_as_float(r[8 * g + 5]) * inv);
+                    w.w = pack2<T>(__uint_as_float(r[8 * g + 6]) * inv, __uint_as_float(r[8 * g + 7]) * inv);
+                    op[g] = w;
+                }
+            }
+        }
+    } else if (tid == 0) {
+        // A bounded wait ran out: record it, let every MMA and copy in flight finish, leave.
+        status_or(p.status, ENERGON_DEVICE_TIMEOUT);
+        umma_commit(drain);
+        mbar_wait_bounded(drain, 0, nullptr, p.timeout_ns);
+        if (q_pending) mbar_wait_bounded(bar_q, 0, nullptr, p.timeout_ns);
+        if (kv_pending) mbar_wait_bounded(bar_kv, kv_parity, nullptr, p.timeout_ns);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, AT_TMEM_COLS);
+}
+
+// ------------------------------------------------------------------ host side
+
+static PFN_cuTensorMapEncodeTiled_v12000 attn_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+bool attention_tc_supported(int dtype, int H, int n_heads, const void* qkv, const void* o, int qkv_rows) {
+    if (dtype != ENERGON_F16 && dtype != ENERGON_BF16) return false;
+    if (n_heads <= 0 || H % n_heads != 0 || H / n_heads != AHD) return false;
+    if (((uintptr_t)qkv | (uintptr_t)o) % 16 != 0 || qkv_rows < 1) return false;
+    return attn_encode_fn() != nullptr;
+}
+
+cudaError_t launch_attention_tc(int dtype, const void* qkv, void* o, const int32_t* cu, int batch, int max_len, int H,
+                                int n_heads, int qkv_rows, int32_t* status, uint64_t timeout_ns, cudaStream_t st) {
+    if (batch <= 0 || max_len <= 0) return cudaSuccess;
+    CUtensorMap tm;
+    cuuint64_t dims[2] = {(cuuint64_t)3 * H, (cuuint64_t)qkv_rows};
+    cuuint64_t strides[1] = {(cuuint64_t)3 * H * 2};
+    cuuint32_t box[2] = {64, 128};
+    cuuint32_t estr[2] = {1, 1};
+    const CUtensorMapDataType dt =
+        dtype == ENERGON_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    CUresult rc = attn_encode_fn()(&tm, dt, 2, const_cast<void*>(qkv), dims, strides, box, estr,
+                                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (rc != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    AttnTcParams p;
+    p.cu = cu;
+    p.out = o;
+    p.status = status;
+    p.H = H;
+    p.scale_log2e = (float)(1.4426950408889634 / sqrt((double)AHD));
+    p.timeout_ns = timeout_ns;
+    dim3 grid((max_len + ATQ - 1) / ATQ, n_heads, batch);
+    if (dtype == ENERGON_BF16) {
+        static bool cfg_b = false;
+        if (!cfg_b) {
+            cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<__nv_bfloat16>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM);
+            if (e != cudaSuccess) return e;
+            cfg_b = true;
+        }
+        attn_tc_kernel<__nv_bfloat16><<<grid, 128, AT_SMEM, st>>>(tm, p);
+    } else {
+        static bool cfg_h = false;
+        if (!cfg_h) {
+            cudaError_t e =
+                cudaFuncSetAttribute(attn_tc_kernel<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM);
+            if (e != cudaSuccess) return e;
+            cfg_h = true;
+        }
+        attn_tc_kernel<__half><<<grid, 128, AT_SMEM, st>>>(tm, p);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace energon

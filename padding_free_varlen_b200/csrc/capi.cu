@@ -208,7 +208,10 @@ int layer_impl(const energon_layer_config& c, const energon_layer_weights& w, co
     if (int r = run_gemm(g, st, "gemm_qkv")) return r;
 
     CK(traced("attention", st,
-              [&] { return launch_attention(c.dtype, ws.qkv, ws.o, cu, batch, max_len, H, c.n_heads, status, st); }),
+              [&] {
+                  return launch_attention(c.dtype, ws.qkv, ws.o, cu, batch, max_len, H, c.n_heads, A_rows, status,
+                                          g_timeout_ns, st);
+              }),
        "attention");
 
     g.A = ws.o, g.W = w.w_o, g.bias = w.b_o, g.residual = x, g.out = ws.x1;

@@ -58,6 +58,7 @@ struct TcParams {
     const int32_t* d_rows;
     int32_t* status;
     int M_cap, N, K, group_m, gelu_tanh;
+    int raster;  // tile order, see tile_coords
     uint64_t timeout_ns;
 };
 
@@ -71,11 +72,33 @@ __device__ __forceinline__ void tile_mn(int t, int num_m, int num_n, int group_m
     m = first_m + (r - n * gm);
 }
 
-// Lane 0 waits, the warp learns the outcome.
+// Tile t -> (m, n).  raster 0: groups of `group` row tiles, columns outermost
+// inside a group (n varies slowest); raster 1: groups of `group` column tiles,
+// rows fastest (every row tile of a column before the next column).
+__device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int group, int raster, int& m, int& n) {
+    if (raster == 0) {
+        tile_mn(t, num_m, num_n, group, m, n);
+        return;
+    }
+    const int per_group = group * num_m;
+    const int g = t / per_group;
+    const int r = t - g * per_group;
+    const int first_n = g * group;
+    const int gn = min(group, num_n - first_n);
+    m = r / gn;
+    n = first_n + (r - m * gn);
+}
+
+// Lane 0 waits, the warp learns the outcome.  SPIN: poll without suspending (the
+// producer and MMA roles, whose wake-up latency stalls the ring); otherwise the
+// suspending wait (the epilogue, which must not steal issue slots from them).
+template <bool SPIN = false>
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const volatile int* abort_flag,
                                           uint64_t timeout_ns) {
     bool ok = true;
-    if ((threadIdx.x & 31) == 0) ok = mbar_wait_bounded(bar, parity, abort_flag, timeout_ns);
+    if ((threadIdx.x & 31) == 0)
+        ok = SPIN ? mbar_spin_bounded(bar, parity, abort_flag, timeout_ns)
+                  : mbar_wait_bounded(bar, parity, abort_flag, timeout_ns);
     return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
@@ -186,9 +209,9 @@ __global__ void __launch_bounds__(256, 1) gemm_tc_kernel(const __grid_constant__
         bool ok = true;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
             int m, n;
-            tile_mn(t, num_m, num_n, p.group_m, m, n);
+            tile_coords(t, num_m, num_n, p.group_m, p.raster, m, n);
             for (int kb = 0; kb < num_kb; ++kb) {
-                if (!warp_wait(&empty[stage], phase ^ 1u, abort_flag, p.timeout_ns)) {
+                if (!warp_wait<true>(&empty[stage], phase ^ 1u, abort_flag, p.timeout_ns)) {
                     ok = false;
                     break;
                 }
@@ -221,14 +244,14 @@ __global__ void __launch_bounds__(256, 1) gemm_tc_kernel(const __grid_constant__
         bool ok = true;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++local) {
             const int acc = local & 1;
-            if (!warp_wait(&tempty[acc], ((local >> 1) & 1) ^ 1, abort_flag, p.timeout_ns)) {
+            if (!warp_wait<true>(&tempty[acc], ((local >> 1) & 1) ^ 1, abort_flag, p.timeout_ns)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
             const uint32_t d_tmem = tmem + (uint32_t)(acc * TBN);
             for (int kb = 0; kb < num_kb; ++kb) {
-                if (!warp_wait(&full[stage], phase, abort_flag, p.timeout_ns)) {
+                if (!warp_wait<true>(&full[stage], phase, abort_flag, p.timeout_ns)) {
                     ok = false;
                     break;
                 }
@@ -270,7 +293,7 @@ __global__ void __launch_bounds__(256, 1) gemm_tc_kernel(const __grid_constant__
             }
             tc_fence_after();
             int m, n;
-            tile_mn(t, num_m, num_n, p.group_m, m, n);
+            tile_coords(t, num_m, num_n, p.group_m, p.raster, m, n);
             const int row = m * TBM + q * 32 + lane;
             const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * TBN);
 #pragma unroll 1
@@ -372,9 +395,9 @@ __global__ void __launch_bounds__(256, 1) gemm_tc2_kernel(const __grid_constant_
         bool ok = true;
         for (int t = pair; t < total && ok; t += npairs) {
             int m, n;
-            tile_mn(t, num_m, num_n, p.group_m, m, n);
+            tile_coords(t, num_m, num_n, p.group_m, p.raster, m, n);
             for (int kb = 0; kb < num_kb; ++kb) {
-                if (!warp_wait(&empty[stage], phase ^ 1u, abort_flag, p.timeout_ns)) {
+                if (!warp_wait<true>(&empty[stage], phase ^ 1u, abort_flag, p.timeout_ns)) {
                     ok = false;
                     break;
                 }
@@ -413,14 +436,14 @@ __global__ void __launch_bounds__(256, 1) gemm_tc2_kernel(const __grid_constant_
         bool ok = true;
         for (int t = pair; t < total && ok; t += npairs, ++local) {
             const int acc = local & 1;
-            if (!warp_wait(&tempty[acc], ((local >> 1) & 1) ^ 1, abort_flag, p.timeout_ns)) {
+            if (!warp_wait<true>(&tempty[acc], ((local >> 1) & 1) ^ 1, abort_flag, p.timeout_ns)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
             const uint32_t d_tmem = tmem + (uint32_t)(acc * PBN);
             for (int kb = 0; kb < num_kb; ++kb) {
-                if (!warp_wait(&full[stage], phase, abort_flag, p.timeout_ns)) {
+                if (!warp_wait<true>(&full[stage], phase, abort_flag, p.timeout_ns)) {
                     ok = false;
                     break;
                 }
@@ -462,7 +485,7 @@ __global__ void __launch_bounds__(256, 1) gemm_tc2_kernel(const __grid_constant_
             }
             tc_fence_after();
             int m, n;
-            tile_mn(t, num_m, num_n, p.group_m, m, n);
+            tile_coords(t, num_m, num_n, p.group_m, p.raster, m, n);
             const int row = m * PBM + (int)rank * 128 + q * 32 + lane;
             const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * PBN);
 #pragma unroll 1
@@ -597,7 +620,7 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st, char* err, size_t
         if (err) snprintf(err, errlen, "cuTensorMapEncodeTiled failed (A: %d, W: %d)", (int)r1, (int)r2);
         return cudaErrorInvalidValue;
     }
-    TcParams p;
+    TcParams p{};
     p.bias = a.bias;
     p.residual = a.residual;
     p.out = a.out;
@@ -611,9 +634,13 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st, char* err, size_t
     const bool bf = a.dtype == ENERGON_BF16;
     if (!single) {
         const int num_m_cap = (a.M_cap + PBM - 1) / PBM, num_n = a.N / PBN;
-        // Raster groups of 8 row tiles (2048 rows): a wave of ~74 pair tiles covers about
-        // 8 x 9 tiles, so each A and W panel is fetched into L2 about once per wave.
-        p.group_m = num_m_cap < 8 ? num_m_cap : 8;
+        // Tile order (measured on the GPT-3 shapes): with up to 16 row tiles every row
+        // tile of a column runs before the next column, so each weight panel is
+        // fetched once while the activation rows (<= 100 MB) stay in L2; with more
+        // rows, one row tile at a time is swept across all columns, keeping its
+        // 6 MB activation panel hot while the weights stream past.
+        p.raster = num_m_cap <= 16 ? 1 : 0;
+        p.group_m = 1;
         const int64_t tiles_cap = (int64_t)num_m_cap * num_n;
         const int pairs = (int)(tiles_cap < device_sm_count() / 2 ? tiles_cap : device_sm_count() / 2);
         switch (a.epilogue) {
@@ -632,6 +659,7 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st, char* err, size_t
     // Rows of A kept hot per raster group: about 48 MiB of the 126 MB L2.
     int gm = (int)((48ll << 20) / ((int64_t)TBM * a.K * 2));
     p.group_m = gm < 1 ? 1 : (gm > num_m_cap ? num_m_cap : gm);
+    p.raster = 0;
     const int64_t tiles_cap = (int64_t)num_m_cap * num_n;
     const int grid = (int)(tiles_cap < device_sm_count() ? tiles_cap : device_sm_count());
     switch (a.epilogue) {

@@ -49,9 +49,14 @@ bool gemm_tc_supported(const GemmArgs& a);
 cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st, char* err, size_t errlen);
 cudaError_t launch_gemm_simt(const GemmArgs& a, cudaStream_t st);
 
-// Causal attention within each sequence: qkv [rows, 3H] -> o [rows, H].
+// Causal attention within each sequence: qkv [rows, 3H] -> o [rows, H].  The
+// tensor-core kernel runs for 16-bit types with head_dim 128 (qkv_rows: rows
+// allocated in qkv, the extent of its tensor map); otherwise the CUDA-core one.
 cudaError_t launch_attention(int dtype, const void* qkv, void* o, const int32_t* cu, int batch, int max_len, int H,
-                             int n_heads, const int32_t* status, cudaStream_t st);
+                             int n_heads, int qkv_rows, int32_t* status, uint64_t timeout_ns, cudaStream_t st);
+bool attention_tc_supported(int dtype, int H, int n_heads, const void* qkv, const void* o, int qkv_rows);
+cudaError_t launch_attention_tc(int dtype, const void* qkv, void* o, const int32_t* cu, int batch, int max_len, int H,
+                                int n_heads, int qkv_rows, int32_t* status, uint64_t timeout_ns, cudaStream_t st);
 
 // Self-test kernel of the bounded wait.
 cudaError_t launch_wait_selftest(int32_t* status, uint64_t timeout_ns, cudaStream_t st);

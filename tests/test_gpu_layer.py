@@ -50,9 +50,9 @@ def step_tol(r: np.ndarray, dtype: int, K: int) -> np.ndarray:
     return ulp(r, dtype) + acc
 
 
-def check_step(name, g, r, dtype, K, report):
+def check_step(name, g, r, dtype, K, report, extra=0.0):
     err = np.abs(g - r)
-    tol = step_tol(r, dtype, K)
+    tol = step_tol(r, dtype, K) + extra
     ratio = float((err / tol).max()) if err.size else 0.0
     report[name] = ratio
     assert ratio <= 1.0, f"{name}: max err/tol {ratio:.3f} (max err {err.max():.3e})"
@@ -104,10 +104,20 @@ def layer_step_checks(res, shape, dtype, oracle_lib):
     flip = np.sqrt(H) * ulp(np.ones(1), dtype)[0] * np.abs(synth.to_f64(w["w_qkv"], dtype)).max() * 0.5
     report["qkv"] = float((err / (step_tol(qkv_ref, dtype, H) + flip)).max())
     assert report["qkv"] <= 1.0, report
-    # attention on the GPU's qkv, one sequence at a time
+    # attention on the GPU's qkv, one sequence at a time.  The tensor-core kernel (16-bit,
+    # head_dim 128) rounds the probabilities P to the storage type before P V: allow
+    # that rounding (unit roundoff times the largest |v| the row can weight).
     o_ref = np.concatenate([oracle_lib.causal_attention(it["qkv"][cu[b]:cu[b + 1]], nh)
                             for b in range(len(cu) - 1)], axis=0)
-    check_step("attention", it["o"], o_ref, dtype, max(1, int(np.diff(cu).max())), report)
+    extra = np.zeros_like(o_ref)
+    if dtype in (synth.F16, synth.BF16) and H // nh == 128:
+        u = 2.0 ** -11 if dtype == synth.F16 else 2.0 ** -8
+        d = H // nh
+        for b in range(len(cu) - 1):
+            v = np.abs(it["qkv"][cu[b]:cu[b + 1], 2 * H:])
+            for j in range(nh):
+                extra[cu[b]:cu[b + 1], j * d:(j + 1) * d] = u * (v[:, j * d:(j + 1) * d].max() if len(v) else 0)
+    check_step("attention", it["o"], o_ref, dtype, max(1, int(np.diff(cu).max())), report, extra)
     check_step("out_proj_residual", it["x1"], x + oracle_lib.linear(it["o"], w["w_o"], w["b_o"]), dtype, H, report)
     check_step("ln2", it["a"], oracle_lib.layernorm(it["x1"], w["ln2_g"], w["ln2_b"]), dtype, H, report)
     check_step("ffn1_gelu", it["f"], oracle_lib.gelu(oracle_lib.linear(it["a"], w["w_1"], w["b_1"])), dtype, H,
