@@ -212,6 +212,30 @@ typedef struct {
 ENERGON_API int energon_trace_start(void);
 ENERGON_API int energon_trace_stop(energon_trace_entry* entries, int capacity, int* n_entries);
 
+/*
+ * transpose_padding_remove for callers that cannot allocate device memory.
+ * The Energon-AI pages have no counterpart to this entry point: it exists for
+ * callers with no cudaMalloc and no workspace at hand, such as an inference
+ * runtime's per-request hook that forbids allocation after start-up, or a
+ * process whose device memory belongs to a pool manager.
+ *   padded, packed, hidden, elem_bytes: as in energon_rce_remove_padding
+ *   lengths   [batch] int32 (device), each in [0, pad_len]
+ *   d_status  int32 out (device): SET as by energon_rce_offsets; with an invalid
+ *             length nothing is gathered
+ * The per-sequence offsets go to a fixed scratch array inside the library image
+ * (present on every GPU that loads the library until the process exits), so
+ * batch may not exceed ENERGON_NOALLOC_MAX_BATCH: larger batches are refused
+ * with ENERGON_ERR_INVALID_ARGUMENT before anything is launched.  The call
+ * allocates nothing.  The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress), so make that first call before any stream
+ * capture.  All calls on a device share the array: calls that may overlap on
+ * the GPU (unordered streams) race; calls ordered on one stream do not.
+ */
+#define ENERGON_NOALLOC_MAX_BATCH 16384
+ENERGON_API int energon_rce_remove_padding_noalloc(const void* padded, const int32_t* lengths, int batch,
+                                                   int pad_len, int hidden, int elem_bytes, void* packed,
+                                                   int32_t* d_status, void* stream);
+
 /* Message describing the last failed call on this thread ("" if none). */
 ENERGON_API const char* energon_last_error(void);
 

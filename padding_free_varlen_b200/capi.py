@@ -35,7 +35,8 @@ DTYPE_OF = {v: k for k, v in TORCH_DTYPE.items()}
 EXPORTED = ("energon_rce_offsets", "energon_rce_remove_padding", "energon_rce_rebuild_padding",
             "energon_workspace_bytes", "energon_layer_forward", "energon_stack_forward",
             "energon_selftest_bounded_wait", "energon_set_wait_timeout_us", "energon_last_error",
-            "energon_trace_start", "energon_trace_stop")
+            "energon_trace_start", "energon_trace_stop", "energon_rce_remove_padding_noalloc")
+ENERGON_NOALLOC_MAX_BATCH = 16384
 WEIGHT_FIELDS = ("ln1_g", "ln1_b", "w_qkv", "b_qkv", "w_o", "b_o",
                  "ln2_g", "ln2_b", "w_1", "b_1", "w_2", "b_2")
 
@@ -82,6 +83,7 @@ def load() -> ctypes.CDLL:
             "energon_set_wait_timeout_us": ([u32], None),
             "energon_last_error": ([], ctypes.c_char_p),
             "energon_trace_start": ([], ci),
+            "energon_rce_remove_padding_noalloc": ([vp, vp, ci, ci, ci, ci, vp, vp, vp], ci),
             "energon_trace_stop": ([ctypes.POINTER(energon_trace_entry), ci, ctypes.POINTER(ci)], ci),
         }
         for name, (args, res) in sigs.items():
@@ -145,6 +147,16 @@ def energon_rce_rebuild_padding(packed, cu_seqlens, batch, pad_len, hidden, elem
     _check(load().energon_rce_rebuild_padding(_dev(packed, "packed"), _dev(cu_seqlens, "cu_seqlens"), batch,
                                               pad_len, hidden, elem_bytes, _dev(padded, "padded"), _stream(stream)),
            "energon_rce_rebuild_padding")
+
+
+def energon_rce_remove_padding_noalloc(padded, lengths, batch, pad_len, hidden, elem_bytes, packed, d_status,
+                                       stream=None) -> None:
+    """Offsets + transpose_padding_remove with the offsets kept in the library's own
+    fixed scratch array: for callers that cannot allocate (batch <= ENERGON_NOALLOC_MAX_BATCH)."""
+    _check(load().energon_rce_remove_padding_noalloc(_dev(padded, "padded"), _dev(lengths, "lengths"), batch, pad_len,
+                                                     hidden, elem_bytes, _dev(packed, "packed"),
+                                                     _dev(d_status, "d_status"), _stream(stream)),
+           "energon_rce_remove_padding_noalloc")
 
 
 def energon_workspace_bytes(cfg: energon_layer_config, batch: int, pad_len: int) -> int:

@@ -236,6 +236,14 @@ int layer_impl(const energon_layer_config& c, const energon_layer_weights& w, co
 
 }  // namespace
 
+namespace energon {
+// Lets the other translation units of the library report through energon_last_error().
+void record_error(int code, const char* msg) {
+    if (code == ENERGON_OK) g_last_error.clear();
+    else g_last_error = msg;
+}
+}  // namespace energon
+
 extern "C" {
 
 const char* energon_last_error(void) { return g_last_error.c_str(); }
