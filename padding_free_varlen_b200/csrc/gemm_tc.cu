@@ -45,10 +45,9 @@ constexpr int TC_SMEM = TSTAGES * (A_STAGE + B_STAGE) + 1024 + 256;
 
 // CTA-pair (cta_group::2) kernel: 256 x 256 tiles, each CTA stages 128 rows of A
 // and 128 rows of W (its half of the tile's N) per 64-wide K step.
-constexpr int PBM = 256, PBN = 256, PBK = 64, PSTAGES = 6;
+constexpr int PBM = 256, PBN = 256, PBK = 64;
 constexpr int PA_STAGE = 128 * PBK * 2;  // 16 KiB
 constexpr int PB_STAGE = 128 * PBK * 2;  // 16 KiB
-constexpr int P_SMEM = PSTAGES * (PA_STAGE + PB_STAGE) + 1024 + 256;
 }  // namespace
 
 struct TcParams {
@@ -329,21 +328,42 @@ __device__ __forceinline__ void spin_ns(uint64_t ns) {
 
 // The CTA-pair variant.  Both CTAs of a 2-CTA cluster load their halves of A
 // (by rows) and W (by the tile's columns) into their own shared memory; the
-// completion of all four copies is counted on the leader CTA's `full` barrier.
-// The leader's MMA thread issues tcgen05.mma.cta_group::2 over both CTAs'
-// shared memory; each CTA receives its 128 accumulator rows in its own TMEM.
-// Commits multicast to both CTAs (ring slots and accumulator hand-off); the
-// peer's epilogue hands accumulators back by arriving on the leader's barrier.
-template <typename T, int EPI>
-__global__ void __launch_bounds__(256, 1) gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA,
-                                                          const __grid_constant__ CUtensorMap tmB, const TcParams p) {
+// completion of every copy is counted on the leader CTA's `full` barrier.  The
+// leader's MMA thread issues tcgen05.mma.cta_group::2 over both CTAs' shared
+// memory; each CTA receives its 128 accumulator rows in its own TMEM.  Commits
+// multicast to both CTAs (ring slots and accumulator hand-off); the peer's
+// epilogue hands accumulators back by arriving on the leader's barrier.
+//
+// MT = row tiles per pair tile.  MT = 1: 256 x 256 tiles, 6-stage ring of 32 KiB
+// per CTA, two 256-column TMEM accumulators so the epilogue of one tile overlaps
+// the MMAs of the next.  MT = 2: 512 x 256 tiles, the staged W panel feeds both
+// row tiles (a quarter less L2 -> SMEM traffic and shared-memory bandwidth per
+// flop), 4-stage ring of 48 KiB, one 512-column accumulator drained by eight
+// epilogue warps between tiles.
+template <int MT>
+struct PairCfg {
+    static constexpr int STAGES = MT == 1 ? 6 : 4;
+    static constexpr int A_STAGE = MT * PA_STAGE;  // MT boxes of 128 rows x 64
+    static constexpr int STAGE = A_STAGE + PB_STAGE;
+    static constexpr int SLOTS = MT == 1 ? 2 : 1;  // TMEM accumulator slots
+    static constexpr int SLOT_COLS = MT * PBN;
+    static constexpr int EPI_WARPS = 4 * MT;
+    static constexpr int THREADS = 128 + 32 * EPI_WARPS;
+    static constexpr int SMEM = STAGES * STAGE + 1024 + 256;
+};
+
+template <typename T, int EPI, int MT>
+__global__ void __launch_bounds__(PairCfg<MT>::THREADS, 1)
+    gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const TcParams p) {
+    using C = PairCfg<MT>;
+    constexpr int NST = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* sA = base;
-    uint8_t* sB = base + PSTAGES * PA_STAGE;
-    uint64_t* full = reinterpret_cast<uint64_t*>(sB + PSTAGES * PB_STAGE);
-    uint64_t* empty = full + PSTAGES;
-    uint64_t* tfull = empty + PSTAGES;
+    uint8_t* sA = base;                    // [stage][MT][128 rows x 128 B]
+    uint8_t* sB = base + NST * C::A_STAGE;  // [stage][128 rows x 128 B]
+    uint64_t* full = reinterpret_cast<uint64_t*>(sB + NST * PB_STAGE);
+    uint64_t* empty = full + NST;
+    uint64_t* tfull = empty + NST;
     uint64_t* tempty = tfull + 2;
     uint64_t* drain = tempty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -357,8 +377,10 @@ __global__ void __launch_bounds__(256, 1) gemm_tc2_kernel(const __grid_constant_
     if (status_bad(p.status)) return;
     const int M = min(*p.d_rows, p.M_cap);
     if (M <= 0) return;
-    const int num_m = (M + PBM - 1) / PBM, num_n = (p.N + PBN - 1) / PBN;
-    const int total = num_m * num_n;
+    const int num_m = (M + PBM - 1) / PBM;               // 256-row tiles
+    const int num_mt = (num_m + MT - 1) / MT;            // pair tiles along M
+    const int num_n = (p.N + PBN - 1) / PBN;
+    const int total = num_mt * num_n;
     if (pair >= total) return;
     const int num_kb = (p.K + PBK - 1) / PBK;
     // Tile order: groups of 8 row tiles (2048 rows); inside a group every row tile of a
@@ -366,16 +388,16 @@ __global__ void __launch_bounds__(256, 1) gemm_tc2_kernel(const __grid_constant_
     // group while the group's activation rows stay in L2.  Measured under sustained load
     // on the four GPT-3 shapes it is within 1 % of every other order tried and ahead of
     // the rest; L2 eviction-priority hints made it 10 % slower.
-    const int raster = 0;
+    const int group = 8 / MT;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < PSTAGES; ++s) {
+        for (int s = 0; s < NST; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull[a], 1);
-            mbar_init(&tempty[a], 8);  // 4 epilogue warps in each CTA of the pair
+            mbar_init(&tempty[a], 2 * C::EPI_WARPS);  // every epilogue warp of both CTAs
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -400,8 +422,8 @@ __global__ void __launch_bounds__(256, 1) gemm_tc2_kernel(const __grid_constant_
         uint32_t phase = 0, pend_mask = 0, pend_par = 0;
         bool ok = true;
         for (int t = pair; t < total && ok; t += npairs) {
-            int m, n;
-            tile_coords(t, num_m, num_n, 8, raster, m, n);
+            int mt, n;
+            tile_coords(t, num_mt, num_n, group, 0, mt, n);
             for (int kb = 0; kb < num_kb; ++kb) {
                 if (!warp_wait<true>(&empty[stage], phase ^ 1u, abort_flag, p.timeout_ns)) {
                     ok = false;
@@ -409,13 +431,16 @@ __global__ void __launch_bounds__(256, 1) gemm_tc2_kernel(const __grid_constant_
                 }
                 if (lane == 0) {
                     const uint32_t bar0 = mapa_shared(smem_u32(&full[stage]), 0);
-                    if (leader) mbar_arrive_expect_tx(&full[stage], 2 * (PA_STAGE + PB_STAGE));
-                    tma_load_2d_pair(sA + stage * PA_STAGE, &tmA, bar0, kb * PBK, m * PBM + (int)rank * 128);
+                    if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE);
+#pragma unroll
+                    for (int i = 0; i < MT; ++i)
+                        tma_load_2d_pair(sA + stage * C::A_STAGE + i * PA_STAGE, &tmA, bar0, kb * PBK,
+                                         (mt * MT + i) * PBM + (int)rank * 128);
                     tma_load_2d_pair(sB + stage * PB_STAGE, &tmB, bar0, kb * PBK, n * PBN + (int)rank * 128);
                 }
                 pend_mask |= 1u << stage;
                 pend_par = (pend_par & ~(1u << stage)) | (phase << stage);
-                if (++stage == PSTAGES) {
+                if (++stage == NST) {
                     stage = 0;
                     phase ^= 1u;
                 }
@@ -425,7 +450,7 @@ __global__ void __launch_bounds__(256, 1) gemm_tc2_kernel(const __grid_constant_
             *abort_flag = 1;
             status_or(p.status, ENERGON_DEVICE_TIMEOUT);
             if (leader) {
-                for (int s = 0; s < PSTAGES; ++s)
+                for (int s = 0; s < NST; ++s)
                     if (pend_mask & (1u << s))
                         mbar_wait_bounded(&full[s], (pend_par >> s) & 1u, nullptr, p.timeout_ns);
             } else {
@@ -441,13 +466,14 @@ __global__ void __launch_bounds__(256, 1) gemm_tc2_kernel(const __grid_constant_
         uint32_t phase = 0;
         bool ok = true;
         for (int t = pair; t < total && ok; t += npairs, ++local) {
-            const int acc = local & 1;
-            if (!warp_wait<true>(&tempty[acc], ((local >> 1) & 1) ^ 1, abort_flag, p.timeout_ns)) {
+            const int slot = local % C::SLOTS;
+            const uint32_t use = (uint32_t)(local / C::SLOTS) & 1u;
+            if (!warp_wait<true>(&tempty[slot], use ^ 1u, abort_flag, p.timeout_ns)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const uint32_t d_tmem = tmem + (uint32_t)(acc * PBN);
+            const uint32_t d_tmem = tmem + (uint32_t)(slot * C::SLOT_COLS);
             for (int kb = 0; kb < num_kb; ++kb) {
                 if (!warp_wait<true>(&full[stage], phase, abort_flag, p.timeout_ns)) {
                     ok = false;
@@ -455,21 +481,26 @@ __global__ void __launch_bounds__(256, 1) gemm_tc2_kernel(const __grid_constant_
                 }
                 tc_fence_after();
                 if (lane == 0) {
-                    const uint64_t a0 = smem_desc_k128(smem_u32(sA + stage * PA_STAGE));
                     const uint64_t b0 = smem_desc_k128(smem_u32(sB + stage * PB_STAGE));
 #pragma unroll
-                    for (int k = 0; k < PBK / 16; ++k)
-                        umma_f16_pair(d_tmem, a0 + 2 * k, b0 + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+                    for (int k = 0; k < PBK / 16; ++k) {
+#pragma unroll
+                        for (int i = 0; i < MT; ++i) {
+                            const uint64_t a0 = smem_desc_k128(smem_u32(sA + stage * C::A_STAGE + i * PA_STAGE));
+                            umma_f16_pair(d_tmem + (uint32_t)(i * PBN), a0 + 2 * k, b0 + 2 * k, idesc,
+                                          (kb | k) != 0 ? 1u : 0u);
+                        }
+                    }
                     umma_commit_pair(&empty[stage], 0x3);
                 }
                 __syncwarp();
-                if (++stage == PSTAGES) {
+                if (++stage == NST) {
                     stage = 0;
                     phase ^= 1u;
                 }
             }
             if (!ok) break;
-            if (lane == 0) umma_commit_pair(&tfull[acc], 0x3);
+            if (lane == 0) umma_commit_pair(&tfull[slot], 0x3);
             __syncwarp();
         }
         if (!ok && lane == 0) {
@@ -480,20 +511,23 @@ __global__ void __launch_bounds__(256, 1) gemm_tc2_kernel(const __grid_constant_
         }
     } else if (warp >= 4) {
         // ---------------------------------------------------------------- epilogue (both CTAs)
-        const int q = warp & 3;
+        const int q = warp & 3;             // TMEM lane quarter this warp may access
+        const int i = (warp - 4) >> 2;      // row tile of the pair tile this warp drains
         int local = 0;
         bool ok = true;
         for (int t = pair; t < total; t += npairs, ++local) {
-            const int acc = local & 1;
-            if (!warp_wait(&tfull[acc], (local >> 1) & 1, abort_flag, p.timeout_ns)) {
+            const int slot = local % C::SLOTS;
+            const uint32_t use = (uint32_t)(local / C::SLOTS) & 1u;
+            if (!warp_wait(&tfull[slot], use, abort_flag, p.timeout_ns)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            int m, n;
-            tile_coords(t, num_m, num_n, 8, raster, m, n);
-            const int row = m * PBM + (int)rank * 128 + q * 32 + lane;
-            const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * PBN);
+            int mt, n;
+            tile_coords(t, num_mt, num_n, group, 0, mt, n);
+            const int row = (mt * MT + i) * PBM + (int)rank * 128 + q * 32 + lane;
+            const uint32_t tbase =
+                tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(slot * C::SLOT_COLS + i * PBN);
 #pragma unroll 1
             for (int c = 0; c < PBN; c += 32) {
                 uint32_t r[32];
@@ -505,7 +539,7 @@ __global__ void __launch_bounds__(256, 1) gemm_tc2_kernel(const __grid_constant_
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
+            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[slot]), 0));
         }
         if (!ok && lane == 0) {
             *abort_flag = 1;
@@ -572,45 +606,52 @@ static cudaError_t tc_launch(const CUtensorMap& ta, const CUtensorMap& tb, const
     return cudaGetLastError();
 }
 
-template <typename T, int EPI>
+template <typename T, int EPI, int MT>
 static cudaError_t tc2_launch(const CUtensorMap& ta, const CUtensorMap& tb, const TcParams& p, int pairs,
                               cudaStream_t st) {
+    using C = PairCfg<MT>;
     static int max_pairs = -1;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
     if (max_pairs < 0) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_tc2_kernel<T, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             P_SMEM);
+        cudaError_t e = cudaFuncSetAttribute(gemm_tc2_kernel<T, EPI, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             C::SMEM);
         if (e != cudaSuccess) return e;
         cudaLaunchConfig_t cfg = {};
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = 2;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
         cfg.gridDim = dim3(2 * (device_sm_count() / 2));
-        cfg.blockDim = dim3(256);
-        cfg.dynamicSmemBytes = P_SMEM;
+        cfg.blockDim = dim3(C::THREADS);
+        cfg.dynamicSmemBytes = C::SMEM;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int clusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&clusters, gemm_tc2_kernel<T, EPI>, &cfg) != cudaSuccess || clusters < 1)
+        if (cudaOccupancyMaxActiveClusters(&clusters, gemm_tc2_kernel<T, EPI, MT>, &cfg) != cudaSuccess ||
+            clusters < 1)
             clusters = device_sm_count() / 2;
         (void)cudaGetLastError();
         max_pairs = clusters;
     }
     if (pairs > max_pairs) pairs = max_pairs;
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
     cfg.gridDim = dim3(2 * pairs);
-    cfg.blockDim = dim3(256);
-    cfg.dynamicSmemBytes = P_SMEM;
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::SMEM;
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<T, EPI>, ta, tb, p);
+    return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<T, EPI, MT>, ta, tb, p);
+}
+
+template <typename T, int MT>
+static cudaError_t tc2_dispatch(int epi, const CUtensorMap& ta, const CUtensorMap& tb, const TcParams& p, int pairs,
+                                cudaStream_t st) {
+    switch (epi) {
+    case EPI_BIAS: return tc2_launch<T, EPI_BIAS, MT>(ta, tb, p, pairs, st);
+    case EPI_BIAS_GELU: return tc2_launch<T, EPI_BIAS_GELU, MT>(ta, tb, p, pairs, st);
+    default: return tc2_launch<T, EPI_BIAS_RESIDUAL, MT>(ta, tb, p, pairs, st);
+    }
 }
 
 // Single-CTA tiles for a GEMM whose rows fit in one 128-row tile (the skinny,
@@ -639,22 +680,19 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st, char* err, size_t
     p.timeout_ns = a.timeout_ns;
     const bool bf = a.dtype == ENERGON_BF16;
     if (!single) {
-        const int num_m_cap = (a.M_cap + PBM - 1) / PBM, num_n = a.N / PBN;
-        p.raster = 0;  // chosen in the kernel from the live row count
+        // Pair tiles of two row tiles (512 x 256) once the buffer can hold two: every
+        // staged weight panel then feeds 512 rows.
+        const int mt = a.M_cap > PBM ? 2 : 1;
+        const int num_m_cap = (a.M_cap + PBM * mt - 1) / (PBM * mt), num_n = a.N / PBN;
+        p.raster = 0;
         p.group_m = 1;
         const int64_t tiles_cap = (int64_t)num_m_cap * num_n;
         const int pairs = (int)(tiles_cap < device_sm_count() / 2 ? tiles_cap : device_sm_count() / 2);
-        switch (a.epilogue) {
-        case EPI_BIAS:
-            return bf ? tc2_launch<__nv_bfloat16, EPI_BIAS>(ta, tb, p, pairs, st)
-                      : tc2_launch<__half, EPI_BIAS>(ta, tb, p, pairs, st);
-        case EPI_BIAS_GELU:
-            return bf ? tc2_launch<__nv_bfloat16, EPI_BIAS_GELU>(ta, tb, p, pairs, st)
-                      : tc2_launch<__half, EPI_BIAS_GELU>(ta, tb, p, pairs, st);
-        default:
-            return bf ? tc2_launch<__nv_bfloat16, EPI_BIAS_RESIDUAL>(ta, tb, p, pairs, st)
-                      : tc2_launch<__half, EPI_BIAS_RESIDUAL>(ta, tb, p, pairs, st);
-        }
+        if (mt == 2)
+            return bf ? tc2_dispatch<__nv_bfloat16, 2>(a.epilogue, ta, tb, p, pairs, st)
+                      : tc2_dispatch<__half, 2>(a.epilogue, ta, tb, p, pairs, st);
+        return bf ? tc2_dispatch<__nv_bfloat16, 1>(a.epilogue, ta, tb, p, pairs, st)
+                  : tc2_dispatch<__half, 1>(a.epilogue, ta, tb, p, pairs, st);
     }
     const int num_m_cap = (a.M_cap + TBM - 1) / TBM, num_n = a.N / TBN;
     // Rows of A kept hot per raster group: about 48 MiB of the 126 MB L2.
