@@ -133,6 +133,8 @@ typedef struct {
  *   a [R, H]   LayerNorm output (after a layer call: the second LayerNorm's)
  *   qkv [R, 3H], o [R, H] (attention output), x1 [R, H] (residual after
  *   attention), f [R, F] (GELU output)      - used by both calls
+ *   p32: fp32 split-K partial sums, 4 * 128 * max(3H, F) floats when
+ *   batch * pad_len <= 128, else 0 bytes        - used by both calls
  *   x [R, H], cu [batch + 1] int32, cu_pad [batch + 1] int32 - stack only
  * After a call completes, the regions hold that call's (last layer's)
  * intermediates for the first T rows, which makes every step inspectable.

@@ -89,8 +89,17 @@ int64_t rows_alloc(int batch, int pad_len) { return (int64_t)align_up((size_t)ba
 
 struct LayerWs {
     void *a, *qkv, *o, *x1, *f;
+    float* p32;  // split-K partial sums (buffers of <= 128 rows only)
+    size_t p32_bytes;
     size_t bytes;
 };
+
+// Split-K scratch for weight-streaming GEMMs: up to 4 splits of 128 rows of the widest output.
+size_t splitk_bytes(const energon_layer_config& c, int batch, int pad_len) {
+    if ((int64_t)batch * pad_len > 128) return 0;
+    const size_t widest = (size_t)(3 * c.hidden > c.ffn ? 3 * c.hidden : c.ffn);
+    return 4 * 128 * widest * sizeof(float);
+}
 
 LayerWs layer_ws_layout(const energon_layer_config& c, int batch, int pad_len, void* base) {
     const size_t e = dtype_bytes(c.dtype);
@@ -109,6 +118,8 @@ LayerWs layer_ws_layout(const energon_layer_config& c, int batch, int pad_len, v
     w.o = take(R * H * e);
     w.x1 = take(R * H * e);
     w.f = take(R * F * e);
+    w.p32_bytes = splitk_bytes(c, batch, pad_len);
+    w.p32 = static_cast<float*>(take(w.p32_bytes));
     w.bytes = off;
     return w;
 }
@@ -202,6 +213,8 @@ int layer_impl(const energon_layer_config& c, const energon_layer_weights& w, co
     g.gelu_tanh = c.gelu_tanh;
     g.status = status;
     g.timeout_ns = g_timeout_ns;
+    g.partials = ws.p32_bytes ? ws.p32 : nullptr;
+    g.partials_bytes = ws.p32_bytes;
 
     g.A = ws.a, g.W = w.w_qkv, g.bias = w.b_qkv, g.residual = nullptr, g.out = ws.qkv;
     g.N = 3 * H, g.K = H, g.epilogue = EPI_BIAS;

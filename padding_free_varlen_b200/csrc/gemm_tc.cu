@@ -57,7 +57,9 @@ struct TcParams {
     const int32_t* d_rows;
     int32_t* status;
     int M_cap, N, K, group_m, gelu_tanh;
-    int raster;  // tile order, see tile_coords
+    int raster;     // tile order, see tile_coords
+    int k_splits;   // single-CTA kernel: K ranges per output tile (1: no split)
+    float* partials;  // k_splits > 1: fp32 [k_splits][M_cap][N] partial sums
     uint64_t timeout_ns;
 };
 
@@ -101,8 +103,11 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
     return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
+// Bias, optional GELU, optional residual (already loaded by the caller into `res`),
+// one rounding to T, 64-byte store of 32 consecutive columns of one row.
 template <typename T, int EPI>
-__device__ __forceinline__ void epilogue_store32(const uint32_t* acc, const TcParams& p, int row, int col0) {
+__device__ __forceinline__ void epilogue_store32(const uint32_t* acc, const uint4* res, const TcParams& p, int row,
+                                                 int col0) {
     float v[32];
 #pragma unroll
     for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(acc[j]);
@@ -121,16 +126,18 @@ __device__ __forceinline__ void epilogue_store32(const uint32_t* acc, const TcPa
         }
     }
     if (EPI == EPI_BIAS_GELU) {
+        if (p.gelu_tanh) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = gelu_f(v[j], p.gelu_tanh != 0);
+            for (int j = 0; j < 32; ++j) v[j] = gelu_tanh_fast(v[j]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = gelu_f(v[j], false);
+        }
     }
-    const int64_t off = (int64_t)row * p.N + col0;
     if (EPI == EPI_BIAS_RESIDUAL) {
-        const uint4* rp = reinterpret_cast<const uint4*>(static_cast<const T*>(p.residual) + off);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            const uint4 w = rp[q];
-            const uint32_t* ww = reinterpret_cast<const uint32_t*>(&w);
+            const uint32_t* ww = reinterpret_cast<const uint32_t*>(&res[q]);
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
                 const float2 f = unpack2<T>(ww[h]);
@@ -139,7 +146,7 @@ __device__ __forceinline__ void epilogue_store32(const uint32_t* acc, const TcPa
             }
         }
     }
-    uint4* op = reinterpret_cast<uint4*>(static_cast<T*>(p.out) + off);
+    uint4* op = reinterpret_cast<uint4*>(static_cast<T*>(p.out) + (int64_t)row * p.N + col0);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         uint4 o;
@@ -148,6 +155,114 @@ __device__ __forceinline__ void epilogue_store32(const uint32_t* acc, const TcPa
         o.z = pack2<T>(v[q * 8 + 4], v[q * 8 + 5]);
         o.w = pack2<T>(v[q * 8 + 6], v[q * 8 + 7]);
         op[q] = o;
+    }
+}
+
+template <typename T, int EPI>
+__device__ __forceinline__ void load_residual32(const TcParams& p, int row, int col0, bool live, uint4* res) {
+    if (EPI == EPI_BIAS_RESIDUAL && live) {
+        const uint4* rp = reinterpret_cast<const uint4*>(static_cast<const T*>(p.residual) + (int64_t)row * p.N + col0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) res[q] = rp[q];
+    }
+}
+
+// One warp drains 256 accumulator columns of its 32 TMEM lanes (= 32 output rows),
+// 32 columns at a time; the TMEM load and the residual load of the next chunk are
+// issued before the current chunk is processed.
+template <typename T, int EPI>
+__device__ __forceinline__ void drain_256(uint32_t tbase, const TcParams& p, int row, int col_base, int M) {
+    uint32_t r[2][32];
+    uint4 res[2][4];
+    const bool row_ok = row < M;
+    tmem_ld_x16(tbase, r[0]);
+    tmem_ld_x16(tbase + 16, r[0] + 16);
+    load_residual32<T, EPI>(p, row, col_base, row_ok && col_base < p.N, res[0]);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        const int cur = c & 1;
+        tmem_wait_ld_regs(r[cur]);
+        if (c + 1 < 8) {
+            tmem_ld_x16(tbase + (c + 1) * 32, r[cur ^ 1]);
+            tmem_ld_x16(tbase + (c + 1) * 32 + 16, r[cur ^ 1] + 16);
+            const int coln = col_base + (c + 1) * 32;
+            load_residual32<T, EPI>(p, row, coln, row_ok && coln < p.N, res[cur ^ 1]);
+        }
+        const int col0 = col_base + c * 32;
+        if (row_ok && col0 < p.N) epilogue_store32<T, EPI>(r[cur], res[cur], p, row, col0);
+    }
+}
+
+// One warp writes its 32 rows x 256 accumulator columns as fp32 partial sums.
+__device__ __forceinline__ void drain_256_partial(uint32_t tbase, float* part, int N, int row, int col_base, int M) {
+#pragma unroll 1
+    for (int c = 0; c < 256; c += 32) {
+        uint32_t r[32];
+        tmem_ld_x16(tbase + c, r);
+        tmem_ld_x16(tbase + c + 16, r + 16);
+        tmem_wait_ld_regs(r);
+        const int col0 = col_base + c;
+        if (row < M && col0 < N) {
+            uint4* dst = reinterpret_cast<uint4*>(part + (int64_t)row * N + col0);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) dst[q] = make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+        }
+    }
+}
+
+// Split-K finish: out[row][col] = epilogue(sum over s = 0 .. S-1 of partials[s][row][col]),
+// the splits summed in index order (deterministic), 8 columns per thread.
+template <typename T, int EPI>
+__global__ void __launch_bounds__(256) splitk_finish_kernel(const float* __restrict__ partials, int S, int M_cap,
+                                                            const int32_t* d_rows, int N, const T* __restrict__ bias,
+                                                            const T* residual, T* out, int gelu_tanh,
+                                                            const int32_t* status) {
+    if (status_bad(status)) return;
+    const int M = min(*d_rows, M_cap);
+    const int vec_per_row = N / 8;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)M * vec_per_row;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int row = (int)(i / vec_per_row), col0 = (int)(i % vec_per_row) * 8;
+        float v[8];
+        const float4* p0 = reinterpret_cast<const float4*>(partials + (int64_t)row * N + col0);
+        float4 a = p0[0], b = p0[1];
+        v[0] = a.x, v[1] = a.y, v[2] = a.z, v[3] = a.w, v[4] = b.x, v[5] = b.y, v[6] = b.z, v[7] = b.w;
+        for (int s = 1; s < S; ++s) {
+            const float4* ps = reinterpret_cast<const float4*>(partials + ((int64_t)s * M_cap + row) * N + col0);
+            a = ps[0], b = ps[1];
+            v[0] += a.x, v[1] += a.y, v[2] += a.z, v[3] += a.w, v[4] += b.x, v[5] += b.y, v[6] += b.z, v[7] += b.w;
+        }
+        if (bias != nullptr) {
+            const uint4 w = *reinterpret_cast<const uint4*>(bias + col0);
+            const uint32_t* ww = reinterpret_cast<const uint32_t*>(&w);
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                const float2 f = unpack2<T>(ww[h]);
+                v[2 * h] += f.x;
+                v[2 * h + 1] += f.y;
+            }
+        }
+        if (EPI == EPI_BIAS_GELU) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[j] = gelu_tanh ? gelu_tanh_fast(v[j]) : gelu_f(v[j], false);
+        }
+        const int64_t off = (int64_t)row * N + col0;
+        if (EPI == EPI_BIAS_RESIDUAL) {
+            const uint4 w = *reinterpret_cast<const uint4*>(residual + off);
+            const uint32_t* ww = reinterpret_cast<const uint32_t*>(&w);
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                const float2 f = unpack2<T>(ww[h]);
+                v[2 * h] += f.x;
+                v[2 * h + 1] += f.y;
+            }
+        }
+        uint4 o;
+        o.x = pack2<T>(v[0], v[1]);
+        o.y = pack2<T>(v[2], v[3]);
+        o.z = pack2<T>(v[4], v[5]);
+        o.w = pack2<T>(v[6], v[7]);
+        *reinterpret_cast<uint4*>(out + off) = o;
     }
 }
 
@@ -171,9 +286,12 @@ __global__ void __launch_bounds__(256, 1) gemm_tc_kernel(const __grid_constant__
     const int M = min(*p.d_rows, p.M_cap);
     if (M <= 0) return;
     const int num_m = (M + TBM - 1) / TBM, num_n = (p.N + TBN - 1) / TBN;
-    const int total = num_m * num_n;
+    // Work unit t = output tile t / S over the K range t % S (S = k_splits, dividing the
+    // K blocks evenly); with S > 1 the epilogue writes fp32 partial sums instead.
+    const int S = p.k_splits;
+    const int total = num_m * num_n * S;
     if ((int)blockIdx.x >= total) return;
-    const int num_kb = (p.K + TBK - 1) / TBK;
+    const int num_kb = (p.K + TBK - 1) / TBK / S;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < TSTAGES; ++s) {
@@ -208,7 +326,8 @@ __global__ void __launch_bounds__(256, 1) gemm_tc_kernel(const __grid_constant__
         bool ok = true;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
             int m, n;
-            tile_coords(t, num_m, num_n, p.group_m, p.raster, m, n);
+            tile_coords(t / S, num_m, num_n, p.group_m, p.raster, m, n);
+            const int kb0 = (t % S) * num_kb;
             for (int kb = 0; kb < num_kb; ++kb) {
                 if (!warp_wait<true>(&empty[stage], phase ^ 1u, abort_flag, p.timeout_ns)) {
                     ok = false;
@@ -216,8 +335,8 @@ __global__ void __launch_bounds__(256, 1) gemm_tc_kernel(const __grid_constant__
                 }
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&full[stage], A_STAGE + B_STAGE);
-                    tma_load_2d(sA + stage * A_STAGE, &tmA, &full[stage], kb * TBK, m * TBM);
-                    tma_load_2d(sB + stage * B_STAGE, &tmB, &full[stage], kb * TBK, n * TBN);
+                    tma_load_2d(sA + stage * A_STAGE, &tmA, &full[stage], (kb0 + kb) * TBK, m * TBM);
+                    tma_load_2d(sB + stage * B_STAGE, &tmB, &full[stage], (kb0 + kb) * TBK, n * TBN);
                 }
                 pend_mask |= 1u << stage;
                 pend_par = (pend_par & ~(1u << stage)) | (phase << stage);
@@ -292,18 +411,13 @@ __global__ void __launch_bounds__(256, 1) gemm_tc_kernel(const __grid_constant__
             }
             tc_fence_after();
             int m, n;
-            tile_coords(t, num_m, num_n, p.group_m, p.raster, m, n);
+            tile_coords(t / S, num_m, num_n, p.group_m, p.raster, m, n);
             const int row = m * TBM + q * 32 + lane;
             const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * TBN);
-#pragma unroll 1
-            for (int c = 0; c < TBN; c += 32) {
-                uint32_t r[32];
-                tmem_ld_x16(tbase + c, r);
-                tmem_ld_x16(tbase + c + 16, r + 16);
-                tmem_wait_ld();
-                const int col0 = n * TBN + c;
-                if (row < M && col0 < p.N) epilogue_store32<T, EPI>(r, p, row, col0);
-            }
+            if (S == 1)
+                drain_256<T, EPI>(tbase, p, row, n * TBN, M);
+            else
+                drain_256_partial(tbase, p.partials + ((int64_t)(t % S) * p.M_cap) * p.N, p.N, row, n * TBN, M);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -528,15 +642,7 @@ __global__ void __launch_bounds__(PairCfg<MT>::THREADS, 1)
             const int row = (mt * MT + i) * PBM + (int)rank * 128 + q * 32 + lane;
             const uint32_t tbase =
                 tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(slot * C::SLOT_COLS + i * PBN);
-#pragma unroll 1
-            for (int c = 0; c < PBN; c += 32) {
-                uint32_t r[32];
-                tmem_ld_x16(tbase + c, r);
-                tmem_ld_x16(tbase + c + 16, r + 16);
-                tmem_wait_ld();
-                const int col0 = n * PBN + c;
-                if (row < M && col0 < p.N) epilogue_store32<T, EPI>(r, p, row, col0);
-            }
+            drain_256<T, EPI>(tbase, p, row, n * PBN, M);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[slot]), 0));
@@ -678,6 +784,8 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st, char* err, size_t
     p.K = a.K;
     p.gelu_tanh = a.gelu_tanh;
     p.timeout_ns = a.timeout_ns;
+    p.k_splits = 1;
+    p.partials = nullptr;
     const bool bf = a.dtype == ENERGON_BF16;
     if (!single) {
         // Pair tiles of two row tiles (512 x 256) once the buffer can hold two: every
@@ -699,19 +807,59 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st, char* err, size_t
     int gm = (int)((48ll << 20) / ((int64_t)TBM * a.K * 2));
     p.group_m = gm < 1 ? 1 : (gm > num_m_cap ? num_m_cap : gm);
     p.raster = 0;
-    const int64_t tiles_cap = (int64_t)num_m_cap * num_n;
-    const int grid = (int)(tiles_cap < device_sm_count() ? tiles_cap : device_sm_count());
+    // Weight-streaming GEMMs with few output tiles split K so that every SM streams:
+    // S minimises (rounds of units over the SMs) / S, e.g. 48 tiles -> 3 splits.
+    const int sms = device_sm_count();
+    const int64_t tiles = (int64_t)num_m_cap * num_n;
+    const int num_kb = a.K / TBK;
+    int S = 1;
+    double best = (double)((tiles + sms - 1) / sms);
+    for (int cand = 2; cand <= 4; ++cand) {
+        if (num_kb % cand != 0) continue;
+        if (a.partials == nullptr || (size_t)cand * a.M_cap * a.N * sizeof(float) > a.partials_bytes) continue;
+        const double cost = (double)((tiles * cand + sms - 1) / sms) / cand;
+        if (cost < best - 1e-9) {
+            best = cost;
+            S = cand;
+        }
+    }
+    p.k_splits = S;
+    p.partials = a.partials;
+    const int64_t units = tiles * S;
+    const int grid = (int)(units < sms ? units : sms);
+    cudaError_t e;
     switch (a.epilogue) {
     case EPI_BIAS:
-        return bf ? tc_launch<__nv_bfloat16, EPI_BIAS>(ta, tb, p, grid, st)
-                  : tc_launch<__half, EPI_BIAS>(ta, tb, p, grid, st);
+        e = bf ? tc_launch<__nv_bfloat16, EPI_BIAS>(ta, tb, p, grid, st) : tc_launch<__half, EPI_BIAS>(ta, tb, p, grid, st);
+        break;
     case EPI_BIAS_GELU:
-        return bf ? tc_launch<__nv_bfloat16, EPI_BIAS_GELU>(ta, tb, p, grid, st)
-                  : tc_launch<__half, EPI_BIAS_GELU>(ta, tb, p, grid, st);
+        e = bf ? tc_launch<__nv_bfloat16, EPI_BIAS_GELU>(ta, tb, p, grid, st)
+               : tc_launch<__half, EPI_BIAS_GELU>(ta, tb, p, grid, st);
+        break;
     default:
-        return bf ? tc_launch<__nv_bfloat16, EPI_BIAS_RESIDUAL>(ta, tb, p, grid, st)
-                  : tc_launch<__half, EPI_BIAS_RESIDUAL>(ta, tb, p, grid, st);
+        e = bf ? tc_launch<__nv_bfloat16, EPI_BIAS_RESIDUAL>(ta, tb, p, grid, st)
+               : tc_launch<__half, EPI_BIAS_RESIDUAL>(ta, tb, p, grid, st);
+        break;
     }
+    if (e != cudaSuccess || S == 1) return e;
+    const int64_t work = (int64_t)a.M_cap * (a.N / 8);
+    const int fgrid = (int)((work + 255) / 256 < 4 * sms ? (work + 255) / 256 : 4 * sms);
+#define FINISH(TT, EE)                                                                                              \
+    splitk_finish_kernel<TT, EE><<<fgrid, 256, 0, st>>>(a.partials, S, a.M_cap, a.d_rows, a.N, (const TT*)a.bias, \
+                                                        (const TT*)a.residual, (TT*)a.out, a.gelu_tanh, a.status)
+    switch (a.epilogue) {
+    case EPI_BIAS:
+        if (bf) FINISH(__nv_bfloat16, EPI_BIAS); else FINISH(__half, EPI_BIAS);
+        break;
+    case EPI_BIAS_GELU:
+        if (bf) FINISH(__nv_bfloat16, EPI_BIAS_GELU); else FINISH(__half, EPI_BIAS_GELU);
+        break;
+    default:
+        if (bf) FINISH(__nv_bfloat16, EPI_BIAS_RESIDUAL); else FINISH(__half, EPI_BIAS_RESIDUAL);
+        break;
+    }
+#undef FINISH
+    return cudaGetLastError();
 }
 
 }  // namespace energon

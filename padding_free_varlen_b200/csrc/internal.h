@@ -37,7 +37,9 @@ struct GemmArgs {
     void* out;                 // [M_cap, N]
     const int32_t* d_rows;     // device: valid rows M (<= M_cap)
     int M_cap, N, K;
-    int A_rows;                // rows allocated in A (>= M_cap; a multiple of 128 for the tensor-core path)
+    int A_rows;                // rows allocated in A (>= M_cap; a multiple of 256 for the tensor-core path)
+    float* partials;           // optional fp32 scratch for split-K of buffers of <= 128 rows
+    size_t partials_bytes;
     int epilogue;
     int gelu_tanh;
     int32_t* status;

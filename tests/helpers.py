@@ -42,6 +42,9 @@ def layer_ws_offsets(H: int, F: int, batch: int, pad_len: int, elem: int) -> dic
     for name, cols in (("a", H), ("qkv", 3 * H), ("o", H), ("x1", H), ("f", F)):
         out[name] = (off, cols)
         off = align_up(off + R * cols * elem, 1024)
+    p32 = 4 * 128 * max(3 * H, F) * 4 if batch * pad_len <= 128 else 0
+    out["p32"] = (off, p32)
+    off = align_up(off + p32, 1024)
     out["_layer_bytes"] = off
     return out
 

@@ -52,11 +52,14 @@ def test_workspace_bytes_matches_documented_layout(lib):
         return (v + a - 1) // a * a
     for (H, nh, F, dt, e, B, S) in [(256, 2, 1024, capi.ENERGON_F16, 2, 3, 70),
                                    (12288, 96, 49152, capi.ENERGON_F16, 2, 32, 256),
+                                   (12288, 96, 49152, capi.ENERGON_F16, 2, 1, 64),
                                    (256, 4, 1024, capi.ENERGON_F32, 4, 4, 32)]:
         R = align(B * S, 256)
         off = 0
-        for cols in (H, 3 * H, H, H, F, H):
+        for cols in (H, 3 * H, H, H, F):
             off = align(off + R * cols * e, 1024)
+        off = align(off + (4 * 128 * max(3 * H, F) * 4 if B * S <= 128 else 0), 1024)   # split-K partials
+        off = align(off + R * H * e, 1024)                                                # stack: x
         off = align(off + (B + 1) * 4, 1024)
         off = align(off + (B + 1) * 4, 1024)
         assert capi.energon_workspace_bytes(cfg(H, nh, F, dt), B, S) == off

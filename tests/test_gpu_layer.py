@@ -193,10 +193,20 @@ def test_stack_packed_equals_padded_and_oracle(oracle_lib, dtype):
         x2[b, :lengths[b]] = x[b, :lengths[b]]
     out2, st3, _ = stack_run(dtype, shape, L, x2, lengths, 12, NONZERO, 1)
     assert st3 == 0 and torch.equal(out2.view(torch.int16), out_pk.view(torch.int16))
-    # a sequence run alone equals its slice of the batch
+    # a sequence run alone equals its slice of the batch: bit for bit when the launch shape
+    # is the same (the other sequences given length 0); as a batch of one, the buffer holds
+    # <= 128 rows and the weight-streaming GEMMs split K, so the sums are ordered
+    # differently and the rows agree within the tolerance instead
     for b in (0, 2):
-        alone, st4, _ = stack_run(dtype, shape, L, x[b:b + 1], lengths[b:b + 1], 12, NONZERO, 1)
-        assert st4 == 0 and torch.equal(alone[0].view(torch.int16), out_pk[b].view(torch.int16))
+        only = np.zeros_like(lengths)
+        only[b] = lengths[b]
+        same_shape, st4, _ = stack_run(dtype, shape, L, x, only, 12, NONZERO, 1)
+        assert st4 == 0 and torch.equal(same_shape[b].view(torch.int16), out_pk[b].view(torch.int16))
+        alone, st5, _ = stack_run(dtype, shape, L, x[b:b + 1], lengths[b:b + 1], 12, NONZERO, 1)
+        assert st5 == 0
+        if lengths[b]:
+            check_end_to_end(to_f64(alone[0, :lengths[b]]), to_f64(out_pk[b, :lengths[b]]), dtype,
+                             f"alone vs batch seq {b}")
 
 
 def test_stack_invalid_lengths_and_empty_batch():
