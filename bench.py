@@ -89,6 +89,11 @@ class Dist:
             dist.destroy_process_group()
 
 
+def replica_value(world: int, tokens_per_step: int, steps: int, ms_max: float) -> float:
+    """Whole-job valid tokens/s of `world` replicas, timed as the slowest rank's duration."""
+    return world * tokens_per_step * steps / (ms_max / 1e3)
+
+
 # ----------------------------------------------------------------------------- clocks
 
 
@@ -333,7 +338,7 @@ def run_energon(args, dist: Dist):
     clk = clocks.stop()
     if int(st.item()) != 0:
         raise RuntimeError(f"device status {int(st.item())} after the timed steps")
-    value = dist.world * T * args.steps / (ms / 1e3)
+    value = replica_value(dist.world, T, args.steps, ms)
 
     # ---- roofline of the dominant kernel (the tcgen05 GEMM, four shapes per layer)
     peaks = load_peaks()
@@ -375,7 +380,7 @@ def run_energon(args, dist: Dist):
         e2e_step()
         torch.cuda.synchronize(dev)
         ms_e2e = timed(e2e_step, args.steps)
-        e2e = {"value": dist.world * T * args.steps / (ms_e2e / 1e3), "unit": UNIT,
+        e2e = {"value": replica_value(dist.world, T, args.steps, ms_e2e), "unit": UNIT,
                "h2d_bytes_per_step": x_host.numel() * x_host.element_size() + len_host.numel() * 4,
                "d2h_bytes_per_step": out_host.numel() * out_host.element_size(),
                "ms_per_step": ms_e2e / args.steps}
@@ -386,7 +391,7 @@ def run_energon(args, dist: Dist):
         kp = max(1, min(args.steps, 3))
         step(0)
         ms_pad = timed(lambda: step(0), kp)
-        padded = {"value": dist.world * T * kp / (ms_pad / 1e3), "unit": UNIT, "ms_per_step": ms_pad / kp,
+        padded = {"value": replica_value(dist.world, T, kp, ms_pad), "unit": UNIT, "ms_per_step": ms_pad / kp,
                   "rows_per_step": B * S, "speedup_of_packed": (ms_pad / kp) / (ms / args.steps)}
 
     launches = sum(v[0] for v in trace.values())
