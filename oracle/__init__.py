@@ -73,6 +73,8 @@ def _L():
             "oracle_offsets": [vp, ci, ci, vp, vp],
             "oracle_remove_padding": [vp, vp, ci, ci, i64, vp],
             "oracle_rebuild_padding": [vp, vp, ci, ci, i64, vp],
+            "oracle_transpose_padding_rebuild": [vp, vp, ci, ci, ci, ci, i64, vp],
+            "oracle_transpose_padding_remove": [vp, vp, ci, ci, ci, ci, i64, vp],
             "oracle_layernorm": [vp, i64, ci, vp, vp, ci, dbl, vp],
             "oracle_linear": [vp, i64, ci, vp, vp, ci, ci, vp],
             "oracle_gelu": [vp, i64, ci, vp],
@@ -142,6 +144,34 @@ def rebuild_padding(packed: np.ndarray, cu: np.ndarray, batch: int, pad_len: int
         out = np.empty((batch, pad_len) + packed.shape[1:], dtype=packed.dtype)
     _check(_L().oracle_rebuild_padding(_ptr(packed), _ptr(cu), batch, pad_len, row_bytes, _ptr(out)),
            "rebuild")
+    return out
+
+
+def transpose_padding_rebuild(packed: np.ndarray, cu: np.ndarray, batch: int, pad_len: int, parts: int,
+                              n_heads: int, out: np.ndarray | None = None) -> np.ndarray:
+    """packed [>=cu[B], parts * n_heads * d] -> head-major [parts, B, n_heads, S, d], zero pads."""
+    packed = np.ascontiguousarray(packed)
+    width = packed.shape[1]
+    assert width % (parts * n_heads) == 0
+    d = width // (parts * n_heads)
+    cu = np.ascontiguousarray(cu, dtype=np.int32)
+    if out is None:
+        out = np.empty((parts, batch, n_heads, pad_len, d), dtype=packed.dtype)
+    _check(_L().oracle_transpose_padding_rebuild(_ptr(packed), _ptr(cu), batch, pad_len, parts, n_heads,
+                                                 d * packed.itemsize, _ptr(out)), "transpose rebuild")
+    return out
+
+
+def transpose_padding_remove(heads: np.ndarray, cu: np.ndarray, out: np.ndarray | None = None) -> np.ndarray:
+    """head-major [parts, B, n_heads, S, d] -> packed [capacity, parts * n_heads * d]
+    (rows >= cu[B] of ``out`` untouched)."""
+    heads = np.ascontiguousarray(heads)
+    parts, B, nh, S, d = heads.shape
+    cu = np.ascontiguousarray(cu, dtype=np.int32)
+    if out is None:
+        out = np.zeros((B * S, parts * nh * d), dtype=heads.dtype)
+    _check(_L().oracle_transpose_padding_remove(_ptr(heads), _ptr(cu), B, S, parts, nh, d * heads.itemsize,
+                                                _ptr(out)), "transpose remove")
     return out
 
 

@@ -134,6 +134,63 @@ int oracle_rebuild_padding(const void* packed, const int32_t* cu, int batch, int
     return 0;
 }
 
+/*
+ * Head-transposing forms of the two operations.  The pages give only the names
+ * transpose_padding_remove / transpose_padding_rebuild ([A] "Runtime"); the
+ * reading for "transpose" is the [token, head] <-> [head, token] exchange a
+ * padded attention stage needs: a packed token row holds `parts` blocks
+ * (1 for an attention output, 3 for Q | K | V) of n_heads heads of
+ * `head_bytes` bytes each, and the head-major padded tensor is
+ * [parts][batch][n_heads][pad_len][head_bytes].
+ *
+ * transpose_padding_rebuild: head-major element (c, b, h, s) is packed row
+ * cu[b] + s, block c, head h, for s < len[b]; all-zero bytes for s >= len[b].
+ */
+int oracle_transpose_padding_rebuild(const void* packed, const int32_t* cu, int batch, int pad_len, int parts,
+                                     int n_heads, int64_t head_bytes, void* heads) {
+    if (!packed || !cu || !heads || batch < 0 || pad_len < 0 || parts < 1 || n_heads < 1 || head_bytes < 0)
+        return 1;
+    const unsigned char* src = (const unsigned char*)packed;
+    unsigned char* dst = (unsigned char*)heads;
+    const int64_t row = (int64_t)parts * n_heads * head_bytes;
+    for (int c = 0; c < parts; ++c)
+        for (int b = 0; b < batch; ++b) {
+            int len = cu[b + 1] - cu[b];
+            for (int h = 0; h < n_heads; ++h)
+                for (int s = 0; s < pad_len; ++s) {
+                    int64_t o = ((((int64_t)c * batch + b) * n_heads + h) * pad_len + s) * head_bytes;
+                    int64_t i = ((int64_t)cu[b] + s) * row + ((int64_t)c * n_heads + h) * head_bytes;
+                    for (int64_t k = 0; k < head_bytes; ++k) dst[o + k] = s < len ? src[i + k] : 0;
+                }
+        }
+    return 0;
+}
+
+/*
+ * transpose_padding_remove: packed row cu[b] + s, block c, head h is head-major
+ * element (c, b, h, s), for every s < len[b]; packed rows at or beyond
+ * cu[batch] are not touched.
+ */
+int oracle_transpose_padding_remove(const void* heads, const int32_t* cu, int batch, int pad_len, int parts,
+                                    int n_heads, int64_t head_bytes, void* packed) {
+    if (!packed || !cu || !heads || batch < 0 || pad_len < 0 || parts < 1 || n_heads < 1 || head_bytes < 0)
+        return 1;
+    const unsigned char* src = (const unsigned char*)heads;
+    unsigned char* dst = (unsigned char*)packed;
+    const int64_t row = (int64_t)parts * n_heads * head_bytes;
+    for (int b = 0; b < batch; ++b) {
+        int len = cu[b + 1] - cu[b];
+        for (int s = 0; s < len; ++s)
+            for (int c = 0; c < parts; ++c)
+                for (int h = 0; h < n_heads; ++h) {
+                    int64_t o = ((int64_t)cu[b] + s) * row + ((int64_t)c * n_heads + h) * head_bytes;
+                    int64_t i = ((((int64_t)c * batch + b) * n_heads + h) * pad_len + s) * head_bytes;
+                    for (int64_t k = 0; k < head_bytes; ++k) dst[o + k] = src[i + k];
+                }
+    }
+    return 0;
+}
+
 /* ----------------------------------------------------------- layer building blocks */
 
 /*

@@ -142,6 +142,72 @@ def test_rebuild_writes_positive_zero(oracle_lib):
     assert out[0, 0].view(np.uint32)[0] == 0x80000000       # valid rows keep their bytes
 
 
+# ----------------------------------------------------------------------------- head-transposing forms
+
+
+def test_transpose_rebuild_remove_hand_case(oracle_lib):
+    # 2 sequences (lengths 2, 1), pad 2, blocks Q|K (parts 2), 2 heads of 1 element;
+    # packed row t holds t*10 + column.  Expected head-major tensor written out by hand.
+    packed = np.array([[t * 10 + j for j in range(4)] for t in range(3)], dtype=np.int16)
+    cu, _ = oracle_lib.offsets(np.array([2, 1]), 2)
+    heads = oracle_lib.transpose_padding_rebuild(packed, cu, 2, 2, parts=2, n_heads=2,
+                                                 out=np.full((2, 2, 2, 2, 1), -1, np.int16))
+    expect = [[[[[0], [10]], [[1], [11]]], [[[20], [0]], [[21], [0]]]],
+              [[[[2], [12]], [[3], [13]]], [[[22], [0]], [[23], [0]]]]]
+    assert heads.tolist() == expect
+    back = oracle_lib.transpose_padding_remove(heads, cu, out=np.full((4, 4), -1, np.int16))
+    assert back[:3].tolist() == packed.tolist() and back[3].tolist() == [-1] * 4
+
+
+def np_transpose_rebuild(packed, lengths, pad_len, parts, nh):
+    """The same map through numpy reshapes and an axis permutation, sequence by sequence."""
+    d = packed.shape[1] // (parts * nh)
+    out = np.zeros((parts, len(lengths), nh, pad_len, d), packed.dtype)
+    r = 0
+    for b, n in enumerate(lengths):
+        out[:, b, :, :n, :] = packed[r:r + n].reshape(n, parts, nh, d).transpose(1, 2, 0, 3)
+        r += n
+    return out
+
+
+@pytest.mark.parametrize("parts,nh,d,dtype", [(3, 4, 8, np.float16), (1, 3, 5, np.float32), (3, 2, 3, np.int8),
+                                              (1, 1, 6, np.uint16)])
+def test_transpose_forms_brute_force(oracle_lib, synth_mod, parts, nh, d, dtype):
+    B, S = 7, 11
+    lengths = synth_mod.uniform_int(B, 0, S, 5, 4)
+    cu, st = oracle_lib.offsets(lengths, S)
+    assert st == 0
+    T, width = int(cu[-1]), parts * nh * d
+    rng = np.random.default_rng(1)
+    isz = np.dtype(dtype).itemsize
+    packed = rng.integers(0, 255, size=(T, width * isz), dtype=np.uint8).view(dtype)
+    heads = oracle_lib.transpose_padding_rebuild(
+        packed, cu, B, S, parts, nh, out=np.full((parts, B, nh, S, d * isz), 0xFF, np.uint8).view(dtype))
+    assert heads.tobytes() == np_transpose_rebuild(packed, lengths, S, parts, nh).tobytes()
+    sentinel = np.full((B * S, width * isz), 0xFF, np.uint8).view(dtype)
+    back = oracle_lib.transpose_padding_remove(heads, cu, out=sentinel)
+    assert back[:T].tobytes() == packed.tobytes()                  # round trip
+    assert (back[T:].view(np.uint8) == 0xFF).all()                 # nothing written past T
+    # remove on a head-major tensor whose pad positions hold garbage ignores them
+    noisy = rng.integers(0, 255, size=heads.view(np.uint8).shape, dtype=np.uint8).view(dtype)
+    got = oracle_lib.transpose_padding_remove(noisy, cu)
+    ref = [noisy[:, b, :, :n, :].transpose(2, 0, 1, 3).reshape(n, width) for b, n in enumerate(lengths)]
+    assert got[:T].tobytes() == np.concatenate(ref).tobytes()
+
+
+def test_transpose_forms_one_block_one_head_are_the_plain_forms(oracle_lib, synth_mod):
+    B, S, H = 5, 9, 12
+    lengths = synth_mod.uniform_int(B, 0, S, 6, 4)
+    cu, _ = oracle_lib.offsets(lengths, S)
+    T = int(cu[-1])
+    packed = synth_mod.normal((T, H), 2, 3, synth_mod.F16)
+    heads = oracle_lib.transpose_padding_rebuild(packed, cu, B, S, 1, 1)
+    assert heads.tobytes() == oracle_lib.rebuild_padding(packed, cu, B, S).tobytes()
+    padded = synth_mod.normal((B, S, H), 2, 4, synth_mod.F16)
+    a = oracle_lib.transpose_padding_remove(padded.reshape(1, B, 1, S, H), cu)
+    assert a[:T].tobytes() == oracle_lib.remove_padding(padded, cu)[:T].tobytes()
+
+
 # ----------------------------------------------------------------------------- decoding
 
 

@@ -23,6 +23,13 @@ MUTANTS = [
      "src[((int64_t)b * len + s) * row_bytes + k]", 1),
     ("rebuild_pads_kept", "? src[((int64_t)cu[b] + s) * row_bytes + k] : 0;",
      "? src[((int64_t)cu[b] + s) * row_bytes + k] : dst[((int64_t)b * pad_len + s) * row_bytes + k];", 1),
+    ("trebuild_block_order", "int64_t i = ((int64_t)cu[b] + s) * row + ((int64_t)c * n_heads + h) * head_bytes;",
+     "int64_t i = ((int64_t)cu[b] + s) * row + ((int64_t)h * parts + c) * head_bytes;", 1),
+    ("trebuild_head_seq_swapped", "int64_t o = ((((int64_t)c * batch + b) * n_heads + h) * pad_len + s) * head_bytes;",
+     "int64_t o = ((((int64_t)c * batch + b) * pad_len + s) * n_heads + h) * head_bytes;", 1),
+    ("trebuild_pads_kept", "dst[o + k] = s < len ? src[i + k] : 0;", "if (s < len) dst[o + k] = src[i + k];", 1),
+    ("tremove_batch_part_swapped", "int64_t i = ((((int64_t)c * batch + b) * n_heads + h) * pad_len + s) * head_bytes;",
+     "int64_t i = ((((int64_t)b * parts + c) * n_heads + h) * pad_len + s) * head_bytes;", 1),
     ("decode_f16_bias", "ldexp((double)(1024 + m), e - 25)", "ldexp((double)(1024 + m), e - 24)", 1),
     ("ln_unbiased_var", "var /= hidden;", "var /= (hidden - 1);", 1),
     ("ln_no_eps", "1.0 / sqrt(var + eps)", "1.0 / sqrt(var)", 1),
