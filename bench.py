@@ -49,6 +49,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-padded", action="store_true")
+    ap.add_argument("--no-transpose", action="store_true")
     ap.add_argument("--layers", type=int, default=0, help="override the workload's layer count (profiling)")
     return ap.parse_args()
 
@@ -393,6 +394,42 @@ def run_energon(args, dist: Dist):
         ms_pad = timed(lambda: step(0), kp)
         padded = {"value": replica_value(dist.world, T, kp, ms_pad), "unit": UNIT, "ms_per_step": ms_pad / kp,
                   "rows_per_step": B * S, "speedup_of_packed": (ms_pad / kp) / (ms / args.steps)}
+        # elimination around each MLP only (attention sub-layers on the padded rows)
+        step(2)
+        ms_mlp = timed(lambda: step(2), kp)
+        padded["mlp_only"] = {"value": replica_value(dist.world, T, kp, ms_mlp), "unit": UNIT,
+                              "ms_per_step": ms_mlp / kp, "speedup_over_padded": ms_pad / ms_mlp}
+
+    # ---- the head-transposing forms on this workload's shapes (Q|K|V rows -> head-major
+    # padded, and an attention output head-major padded -> packed rows)
+    transpose = None
+    if not args.no_transpose and H % wl.shape.n_heads == 0:
+        nh = wl.shape.n_heads
+        d = H // nh
+        qkv_rows = torch.zeros((T, 3 * H), dtype=tdt, device=dev)
+        heads = torch.empty((3, B, nh, S, d), dtype=tdt, device=dev)
+        back = torch.empty((T, H), dtype=tdt, device=dev)
+        cu_dev = torch.empty(B + 1, dtype=torch.int32, device=dev)
+        capi.energon_rce_offsets(d_len, B, S, cu_dev, st, stream)
+        kt = max(3, args.steps)
+
+        def t_rebuild():
+            capi.energon_rce_transpose_padding_rebuild(qkv_rows, cu_dev, B, S, 3, nh, d, e, heads, stream)
+
+        def t_remove():
+            capi.energon_rce_transpose_padding_remove(heads, cu_dev, B, S, 1, nh, d, e, back, stream)
+        transpose = {}
+        for name, fn, nbytes in (("transpose_padding_rebuild_qkv", t_rebuild, T * 3 * H * e + 3 * B * S * H * e),
+                                 ("transpose_padding_remove_attn", t_remove, 2 * T * H * e)):
+            fn()
+            ms_t = timed(fn, kt) / kt
+            gbs = nbytes / (ms_t / 1e3) / 1e9
+            transpose[name] = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                               "frac": gbs / peaks["hbm_gbs"], "algorithmic_bytes_per_launch": nbytes,
+                               "ms_per_launch": ms_t}
+        del qkv_rows, heads, back
+        if int(st.item()) != 0:
+            raise RuntimeError(f"device status {int(st.item())} after the transpose forms")
 
     launches = sum(v[0] for v in trace.values())
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": dist.world, "steps": args.steps,
@@ -401,7 +438,7 @@ def run_energon(args, dist: Dist):
             "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights)",
             "config": config_of(wl, S, T, dist.world), "roofline": roofline, "roofline_memory_kernels": aux,
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clk,
-            "padded_path": padded, "kernels": per_kernel, "setup_s": setup_s}
+            "padded_path": padded, "transpose_forms": transpose, "kernels": per_kernel, "setup_s": setup_s}
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
     del tables

@@ -107,6 +107,34 @@ ENERGON_API int energon_rce_rebuild_padding(const void* packed, const int32_t* c
                                 int pad_len, int hidden, int elem_bytes, void* padded,
                                 void* stream);
 
+/*
+ * Head-transposing forms of the two operations above (QbitAI article, "Runtime",
+ * which names transpose_padding_rebuild / transpose_padding_remove and nothing
+ * more; the "transpose" is read as the [token, head] <-> [head, token] exchange
+ * that an attention stage on the padded, head-major layout needs).
+ *   packed      [>= T, parts * n_heads * head_dim]: a token row holds `parts`
+ *               blocks (1 for an attention output, 3 for Q | K | V), each of
+ *               n_heads heads of head_dim elements of elem_bytes bytes
+ *   heads       [parts, batch, n_heads, pad_len, head_dim]
+ *   cu_seqlens  [batch + 1] from energon_rce_offsets (device)
+ * transpose_padding_rebuild writes EVERY element of `heads`: (c, b, h, s, :) is
+ * block c, head h of packed row cu[b] + s when s < len[b], all-zero bytes
+ * otherwise.  transpose_padding_remove writes packed rows 0 .. T-1 only: row
+ * cu[b] + s, block c, head h receives heads (c, b, h, s, :); pad positions of
+ * `heads` are never read.  Byte copies (bit-exact).  elem_bytes in {1, 2, 4, 8};
+ * parts >= 1, n_heads >= 1, head_dim >= 0, parts * n_heads * head_dim *
+ * elem_bytes < 2^31; any pointer alignment (16-byte vector path when head_dim *
+ * elem_bytes and both pointers allow it).  The buffers are the caller's;
+ * nothing is allocated.  Errors: NULL pointer, negative size or a bad
+ * elem_bytes -> ENERGON_ERR_INVALID_ARGUMENT before any launch.
+ */
+ENERGON_API int energon_rce_transpose_padding_rebuild(const void* packed, const int32_t* cu_seqlens, int batch,
+                                          int pad_len, int parts, int n_heads, int head_dim, int elem_bytes,
+                                          void* heads, void* stream);
+ENERGON_API int energon_rce_transpose_padding_remove(const void* heads, const int32_t* cu_seqlens, int batch,
+                                         int pad_len, int parts, int n_heads, int head_dim, int elem_bytes,
+                                         void* packed, void* stream);
+
 /* Weights of one pre-LN GPT decoder layer, all of the config's dtype, device:
  *   ln1_g, ln1_b [H]; w_qkv [3H, H], b_qkv [3H] (output columns Q | K | V, each
  *   head-major); w_o [H, H], b_o [H]; ln2_g, ln2_b [H]; w_1 [F, H], b_1 [F];
@@ -171,7 +199,11 @@ ENERGON_API int energon_layer_forward(const energon_layer_config* cfg, const ene
  *   remove_padding 1: run the layers on the T valid tokens (the service
  *                  config's rm_padding = True in the QbitAI article's usability
  *                  example); 0: run them on all batch * pad_len rows (the padded
- *                  baseline the pages compare against), valid rows unchanged.
+ *                  baseline the pages compare against); 2: eliminate the padding
+ *                  in the MLP only, as the article's "Runtime" section states
+ *                  it - each layer's attention sub-layer on all rows, then
+ *                  remove, the MLP on the valid tokens, rebuild.  Valid rows are
+ *                  the same in all three modes.
  *   padded_out    [batch, pad_len, H]: valid rows hold the stack's output, pad
  *                 rows are zero.  With invalid lengths: all zero, d_status = 1.
  *   d_status      required; SET by the offsets step, then OR-ed by later kernels.

@@ -35,7 +35,8 @@ DTYPE_OF = {v: k for k, v in TORCH_DTYPE.items()}
 EXPORTED = ("energon_rce_offsets", "energon_rce_remove_padding", "energon_rce_rebuild_padding",
             "energon_workspace_bytes", "energon_layer_forward", "energon_stack_forward",
             "energon_selftest_bounded_wait", "energon_set_wait_timeout_us", "energon_last_error",
-            "energon_trace_start", "energon_trace_stop", "energon_rce_remove_padding_noalloc")
+            "energon_trace_start", "energon_trace_stop", "energon_rce_remove_padding_noalloc",
+            "energon_rce_transpose_padding_rebuild", "energon_rce_transpose_padding_remove")
 ENERGON_NOALLOC_MAX_BATCH = 16384
 WEIGHT_FIELDS = ("ln1_g", "ln1_b", "w_qkv", "b_qkv", "w_o", "b_o",
                  "ln2_g", "ln2_b", "w_1", "b_1", "w_2", "b_2")
@@ -76,6 +77,8 @@ def load() -> ctypes.CDLL:
             "energon_rce_offsets": ([vp, ci, ci, vp, vp, vp], ci),
             "energon_rce_remove_padding": ([vp, vp, ci, ci, ci, ci, vp, vp], ci),
             "energon_rce_rebuild_padding": ([vp, vp, ci, ci, ci, ci, vp, vp], ci),
+            "energon_rce_transpose_padding_rebuild": ([vp, vp, ci, ci, ci, ci, ci, ci, vp, vp], ci),
+            "energon_rce_transpose_padding_remove": ([vp, vp, ci, ci, ci, ci, ci, ci, vp, vp], ci),
             "energon_workspace_bytes": ([cfgp, ci, ci], sz),
             "energon_layer_forward": ([cfgp, wp, vp, vp, ci, ci, vp, vp, vp, sz, vp], ci),
             "energon_stack_forward": ([cfgp, wp, ci, vp, vp, ci, ci, ci, vp, vp, vp, sz, vp], ci),
@@ -147,6 +150,22 @@ def energon_rce_rebuild_padding(packed, cu_seqlens, batch, pad_len, hidden, elem
     _check(load().energon_rce_rebuild_padding(_dev(packed, "packed"), _dev(cu_seqlens, "cu_seqlens"), batch,
                                               pad_len, hidden, elem_bytes, _dev(padded, "padded"), _stream(stream)),
            "energon_rce_rebuild_padding")
+
+
+def energon_rce_transpose_padding_rebuild(packed, cu_seqlens, batch, pad_len, parts, n_heads, head_dim, elem_bytes,
+                                          heads, stream=None) -> None:
+    _check(load().energon_rce_transpose_padding_rebuild(_dev(packed, "packed"), _dev(cu_seqlens, "cu_seqlens"), batch,
+                                                        pad_len, parts, n_heads, head_dim, elem_bytes,
+                                                        _dev(heads, "heads"), _stream(stream)),
+           "energon_rce_transpose_padding_rebuild")
+
+
+def energon_rce_transpose_padding_remove(heads, cu_seqlens, batch, pad_len, parts, n_heads, head_dim, elem_bytes,
+                                         packed, stream=None) -> None:
+    _check(load().energon_rce_transpose_padding_remove(_dev(heads, "heads"), _dev(cu_seqlens, "cu_seqlens"), batch,
+                                                       pad_len, parts, n_heads, head_dim, elem_bytes,
+                                                       _dev(packed, "packed"), _stream(stream)),
+           "energon_rce_transpose_padding_remove")
 
 
 def energon_rce_remove_padding_noalloc(padded, lengths, batch, pad_len, hidden, elem_bytes, packed, d_status,

@@ -193,58 +193,71 @@ int run_gemm(GemmArgs& g, cudaStream_t st, const char* what) {
     return ENERGON_OK;
 }
 
-// One layer; cu = row starts of the sequences (device), rows valid = cu[batch].
-int layer_impl(const energon_layer_config& c, const energon_layer_weights& w, const void* x, const int32_t* cu,
-               int batch, int max_len, void* y, int32_t* status, const LayerWs& ws, cudaStream_t st) {
-    const int H = c.hidden, F = c.ffn;
-    const int M_cap = batch * max_len;
-    const int A_rows = (int)rows_alloc(batch, max_len);
-    const int32_t* d_rows = cu + batch;
-
-    CK(traced("layernorm", st,
-              [&] { return launch_layernorm(c.dtype, x, w.ln1_g, w.ln1_b, ws.a, d_rows, M_cap, H, c.ln_eps, status, st); }),
-       "ln1");
-
+GemmArgs gemm_base(const energon_layer_config& c, const int32_t* cu, int batch, int max_len, int32_t* status,
+                   const LayerWs& ws) {
     GemmArgs g{};
     g.dtype = c.dtype;
-    g.d_rows = d_rows;
-    g.M_cap = M_cap;
-    g.A_rows = A_rows;
+    g.d_rows = cu + batch;
+    g.M_cap = batch * max_len;
+    g.A_rows = (int)rows_alloc(batch, max_len);
     g.gelu_tanh = c.gelu_tanh;
     g.status = status;
     g.timeout_ns = g_timeout_ns;
     g.partials = ws.p32_bytes ? ws.p32 : nullptr;
     g.partials_bytes = ws.p32_bytes;
+    return g;
+}
 
+// Attention sub-layer on the rows described by cu (row starts; rows valid = cu[batch]):
+//   x1 = x + attention(LN1(x) W_qkv^T + b_qkv) W_o^T + b_o
+int attention_sublayer(const energon_layer_config& c, const energon_layer_weights& w, const void* x,
+                       const int32_t* cu, int batch, int max_len, void* x1, int32_t* status, const LayerWs& ws,
+                       cudaStream_t st) {
+    const int H = c.hidden;
+    const int M_cap = batch * max_len;
+    const int A_rows = (int)rows_alloc(batch, max_len);
+    const int32_t* d_rows = cu + batch;
+    CK(traced("layernorm", st,
+              [&] { return launch_layernorm(c.dtype, x, w.ln1_g, w.ln1_b, ws.a, d_rows, M_cap, H, c.ln_eps, status, st); }),
+       "ln1");
+    GemmArgs g = gemm_base(c, cu, batch, max_len, status, ws);
     g.A = ws.a, g.W = w.w_qkv, g.bias = w.b_qkv, g.residual = nullptr, g.out = ws.qkv;
     g.N = 3 * H, g.K = H, g.epilogue = EPI_BIAS;
     if (int r = run_gemm(g, st, "gemm_qkv")) return r;
-
     CK(traced("attention", st,
               [&] {
                   return launch_attention(c.dtype, ws.qkv, ws.o, cu, batch, max_len, H, c.n_heads, A_rows, status,
                                           g_timeout_ns, st);
               }),
        "attention");
-
-    g.A = ws.o, g.W = w.w_o, g.bias = w.b_o, g.residual = x, g.out = ws.x1;
+    g.A = ws.o, g.W = w.w_o, g.bias = w.b_o, g.residual = x, g.out = x1;
     g.N = H, g.K = H, g.epilogue = EPI_BIAS_RESIDUAL;
-    if (int r = run_gemm(g, st, "gemm_out_proj")) return r;
+    return run_gemm(g, st, "gemm_out_proj");
+}
 
+// MLP sub-layer: y = x1 + GELU(LN2(x1) W_1^T + b_1) W_2^T + b_2 (y may alias nothing but itself).
+int mlp_sublayer(const energon_layer_config& c, const energon_layer_weights& w, const void* x1, const int32_t* cu,
+                 int batch, int max_len, void* y, int32_t* status, const LayerWs& ws, cudaStream_t st) {
+    const int H = c.hidden, F = c.ffn;
+    const int M_cap = batch * max_len;
+    const int32_t* d_rows = cu + batch;
     CK(traced("layernorm", st,
-              [&] {
-                  return launch_layernorm(c.dtype, ws.x1, w.ln2_g, w.ln2_b, ws.a, d_rows, M_cap, H, c.ln_eps, status, st);
-              }),
+              [&] { return launch_layernorm(c.dtype, x1, w.ln2_g, w.ln2_b, ws.a, d_rows, M_cap, H, c.ln_eps, status, st); }),
        "ln2");
-
+    GemmArgs g = gemm_base(c, cu, batch, max_len, status, ws);
     g.A = ws.a, g.W = w.w_1, g.bias = w.b_1, g.residual = nullptr, g.out = ws.f;
     g.N = F, g.K = H, g.epilogue = EPI_BIAS_GELU;
     if (int r = run_gemm(g, st, "gemm_ffn1")) return r;
-
-    g.A = ws.f, g.W = w.w_2, g.bias = w.b_2, g.residual = ws.x1, g.out = y;
+    g.A = ws.f, g.W = w.w_2, g.bias = w.b_2, g.residual = x1, g.out = y;
     g.N = H, g.K = F, g.epilogue = EPI_BIAS_RESIDUAL;
-    if (int r = run_gemm(g, st, "gemm_ffn2")) return r;
-    return ENERGON_OK;
+    return run_gemm(g, st, "gemm_ffn2");
+}
+
+// One layer; cu = row starts of the sequences (device), rows valid = cu[batch].
+int layer_impl(const energon_layer_config& c, const energon_layer_weights& w, const void* x, const int32_t* cu,
+               int batch, int max_len, void* y, int32_t* status, const LayerWs& ws, cudaStream_t st) {
+    if (int r = attention_sublayer(c, w, x, cu, batch, max_len, ws.x1, status, ws, st)) return r;
+    return mlp_sublayer(c, w, ws.x1, cu, batch, max_len, y, status, ws, st);
 }
 
 }  // namespace
@@ -301,6 +314,46 @@ int energon_rce_rebuild_padding(const void* packed, const int32_t* cu_seqlens, i
     return ENERGON_OK;
 }
 
+static int check_head_form(const char* what, const void* a, const void* b, const int32_t* cu, int batch,
+                           int pad_len, int parts, int n_heads, int head_dim, int elem_bytes) {
+    if (!a || !b || !cu) return fail(ENERGON_ERR_INVALID_ARGUMENT, "%s: NULL pointer", what);
+    if (batch < 0 || pad_len < 0 || head_dim < 0 || parts < 1 || n_heads < 1)
+        return fail(ENERGON_ERR_INVALID_ARGUMENT, "%s: negative size, or parts / n_heads below 1", what);
+    if (elem_bytes != 1 && elem_bytes != 2 && elem_bytes != 4 && elem_bytes != 8)
+        return fail(ENERGON_ERR_INVALID_ARGUMENT, "%s: elem_bytes must be 1, 2, 4 or 8", what);
+    if ((int64_t)parts * n_heads * head_dim * elem_bytes > (int64_t)0x7fffffff)
+        return fail(ENERGON_ERR_INVALID_ARGUMENT, "%s: packed row of 2^31 bytes or more", what);
+    if ((int64_t)batch * pad_len > (int64_t)0x7fffff00)
+        return fail(ENERGON_ERR_INVALID_ARGUMENT, "%s: batch * pad_len exceeds the int32 token index", what);
+    return ENERGON_OK;
+}
+
+int energon_rce_transpose_padding_rebuild(const void* packed, const int32_t* cu_seqlens, int batch, int pad_len,
+                                          int parts, int n_heads, int head_dim, int elem_bytes, void* heads,
+                                          void* stream) {
+    g_last_error.clear();
+    if (int r = check_head_form("transpose rebuild", packed, heads, cu_seqlens, batch, pad_len, parts, n_heads,
+                                head_dim, elem_bytes))
+        return r;
+    CK(launch_transpose_rebuild(packed, cu_seqlens, batch, pad_len, parts, n_heads, (int64_t)head_dim * elem_bytes,
+                                (int64_t)batch * pad_len, heads, (cudaStream_t)stream),
+       "transpose rebuild");
+    return ENERGON_OK;
+}
+
+int energon_rce_transpose_padding_remove(const void* heads, const int32_t* cu_seqlens, int batch, int pad_len,
+                                         int parts, int n_heads, int head_dim, int elem_bytes, void* packed,
+                                         void* stream) {
+    g_last_error.clear();
+    if (int r = check_head_form("transpose remove", heads, packed, cu_seqlens, batch, pad_len, parts, n_heads,
+                                head_dim, elem_bytes))
+        return r;
+    CK(launch_transpose_remove(heads, cu_seqlens, batch, pad_len, parts, n_heads, (int64_t)head_dim * elem_bytes,
+                               (int64_t)batch * pad_len, packed, (cudaStream_t)stream),
+       "transpose remove");
+    return ENERGON_OK;
+}
+
 size_t energon_workspace_bytes(const energon_layer_config* cfg, int batch, int pad_len) {
     if (check_config(cfg) != ENERGON_OK || check_sizes(batch, pad_len) != ENERGON_OK) return 0;
     return stack_ws_layout(*cfg, batch, pad_len, nullptr).bytes;
@@ -333,6 +386,8 @@ int energon_stack_forward(const energon_layer_config* cfg, const energon_layer_w
     if (!padded_in || !lengths || !padded_out || !d_status || !workspace)
         return fail(ENERGON_ERR_INVALID_ARGUMENT, "stack: NULL pointer");
     if (padded_in == padded_out) return fail(ENERGON_ERR_INVALID_ARGUMENT, "stack: padded_out aliases padded_in");
+    if (remove_padding < 0 || remove_padding > 2)
+        return fail(ENERGON_ERR_INVALID_ARGUMENT, "stack: remove_padding must be 0, 1 or 2");
     const StackWs ws = stack_ws_layout(*cfg, batch, pad_len, workspace);
     if (ws_bytes < ws.bytes)
         return fail(ENERGON_ERR_WORKSPACE_TOO_SMALL, "stack: workspace %zu < %zu bytes", ws_bytes, ws.bytes);
@@ -342,7 +397,7 @@ int energon_stack_forward(const energon_layer_config* cfg, const energon_layer_w
 
     CK(traced("offsets", st, [&] { return launch_offsets(lengths, batch, pad_len, ws.cu, d_status, st); }),
        "offsets");
-    if (remove_padding) {
+    if (remove_padding == 1) {
         CK(traced("remove_padding", st,
                   [&] { return launch_remove(padded_in, ws.cu, batch, pad_len, row_bytes, ws.x, R, d_status, st); }),
            "remove");
@@ -352,6 +407,40 @@ int energon_stack_forward(const energon_layer_config* cfg, const energon_layer_w
         CK(traced("rebuild_padding", st,
                   [&] { return launch_rebuild(ws.x, ws.cu, ws.cu, batch, pad_len, row_bytes, R, padded_out, st); }),
            "rebuild");
+    } else if (remove_padding == 2) {
+        // Elimination for the MLP only, as the QbitAI article's "Runtime" section states it:
+        // each layer's attention sub-layer runs on all batch * pad_len rows; its output is
+        // packed (remove), the MLP sub-layer runs on the valid tokens, and the result is
+        // scattered back (rebuild, zero pads) for the next layer.
+        CK(traced("padded_starts", st, [&] { return launch_padded_starts(batch, pad_len, ws.cu_pad, d_status, st); }),
+           "padded starts");
+        const void* src = padded_in;
+        void* x1_pk = ws.layer.o;    // free once the out-projection has consumed it
+        void* y_pk = ws.layer.qkv;   // free once attention has consumed it
+        for (int l = 0; l < n_layers; ++l) {
+            if (int r = attention_sublayer(*cfg, layers[l], src, ws.cu_pad, batch, pad_len, ws.layer.x1, d_status,
+                                           ws.layer, st))
+                return r;
+            CK(traced("remove_padding", st,
+                      [&] {
+                          return launch_remove(ws.layer.x1, ws.cu, batch, pad_len, row_bytes, x1_pk, R, d_status, st);
+                      }),
+               "remove");
+            if (int r = mlp_sublayer(*cfg, layers[l], x1_pk, ws.cu, batch, pad_len, y_pk, d_status, ws.layer, st))
+                return r;
+            void* dst = (l + 1 == n_layers) ? padded_out : ws.x;
+            CK(traced("rebuild_padding", st,
+                      [&] { return launch_rebuild(y_pk, ws.cu, ws.cu, batch, pad_len, row_bytes, R, dst, st); }),
+               "rebuild");
+            src = ws.x;
+        }
+        if (n_layers == 0)
+            CK(traced("rebuild_padding", st,
+                      [&] {
+                          return launch_rebuild(padded_in, ws.cu_pad, ws.cu, batch, pad_len, row_bytes, R, padded_out,
+                                                st);
+                      }),
+               "rebuild");
     } else {
         // Padded baseline: every one of the batch * pad_len rows goes through the layers.
         CK(traced("padded_starts", st, [&] { return launch_padded_starts(batch, pad_len, ws.cu_pad, d_status, st); }),

@@ -20,6 +20,14 @@ cudaError_t launch_remove(const void* padded, const int32_t* cu, int batch, int 
 // len_b = lens_cu[b+1] - lens_cu[b].  Writes every padded row.
 cudaError_t launch_rebuild(const void* packed, const int32_t* starts, const int32_t* lens_cu, int batch,
                            int pad_len, int64_t row_bytes, int64_t packed_rows_cap, void* padded, cudaStream_t st);
+// Head-transposing forms: packed rows of `parts` blocks of n_heads heads of
+// head_bytes bytes <-> head-major [parts][batch][n_heads][pad_len][head_bytes].
+cudaError_t launch_transpose_rebuild(const void* packed, const int32_t* cu, int batch, int pad_len, int parts,
+                                     int n_heads, int64_t head_bytes, int64_t packed_rows_cap, void* heads,
+                                     cudaStream_t st);
+cudaError_t launch_transpose_remove(const void* heads, const int32_t* cu, int batch, int pad_len, int parts,
+                                    int n_heads, int64_t head_bytes, int64_t packed_rows_cap, void* packed,
+                                    cudaStream_t st);
 
 // LayerNorm over rows [0, min(*d_rows, rows_cap)) of x [rows_cap, H] -> y.
 cudaError_t launch_layernorm(int dtype, const void* x, const void* g, const void* b, void* y, const int32_t* d_rows,

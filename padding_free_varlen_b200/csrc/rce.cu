@@ -215,6 +215,168 @@ cudaError_t launch_rebuild(const void* packed, const int32_t* starts, const int3
     return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ head-transposing forms
+//
+// A packed token row holds `parts` blocks of n_heads heads of head_vecs vectors;
+// the head-major padded tensor is [parts][batch][n_heads][pad_len][head_vecs].
+// One warp per row (a padded position for rebuild, a packed token for remove):
+// consecutive lanes walk the packed row, so its reads (rebuild) or writes
+// (remove) are contiguous, and each head's run of head_vecs vectors lands in one
+// contiguous segment of the head-major tensor.
+
+struct HeadMap {
+    int n_heads, head_vecs, row_vecs;  // row_vecs = parts * n_heads * head_vecs
+    int batch, pad_len;
+    int step_blk, step_j;              // 32 vectors = step_blk whole heads + step_j vectors
+};
+
+// Walks the vectors lane, lane + 32, lane + 64, ... of one packed row and keeps
+// their head coordinates (block c, head h, vector j) up to date by addition, so
+// the per-vector cost is a few integer adds instead of two divisions.
+struct HeadCursor {
+    int c, h, j;
+    __device__ __forceinline__ HeadCursor(const HeadMap& m, int lane) {
+        const int blk = lane / m.head_vecs;
+        j = lane - blk * m.head_vecs;
+        c = blk / m.n_heads;
+        h = blk - c * m.n_heads;
+    }
+    __device__ __forceinline__ void advance(const HeadMap& m) {
+        j += m.step_j;
+        int dh = m.step_blk;
+        if (j >= m.head_vecs) j -= m.head_vecs, ++dh;
+        h += dh;
+        while (h >= m.n_heads) h -= m.n_heads, ++c;  // at most step_blk / n_heads + 1 turns
+    }
+    // head-major offset (in vectors) of this vector at position (b, s)
+    __device__ __forceinline__ int64_t offset(const HeadMap& m, int b, int s) const {
+        return ((((int64_t)c * m.batch + b) * m.n_heads + h) * m.pad_len + s) * m.head_vecs + j;
+    }
+};
+
+template <typename V, int UNROLL>
+__global__ void __launch_bounds__(256) transpose_rebuild_kernel(const V* __restrict__ packed,
+                                                                const int32_t* __restrict__ cu, HeadMap m,
+                                                                int64_t packed_rows_cap, V* __restrict__ heads) {
+    const int lane = threadIdx.x & 31;
+    const int64_t rows = (int64_t)m.batch * m.pad_len;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    V z;
+    memset(&z, 0, sizeof(V));
+    for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
+        const int b = (int)(r / m.pad_len);
+        const int s = (int)(r - (int64_t)b * m.pad_len);
+        const int len = __ldg(cu + b + 1) - __ldg(cu + b);
+        const int64_t src = (int64_t)__ldg(cu + b) + s;
+        const bool valid = s < len && src >= 0 && src < packed_rows_cap;
+        const V* row = packed + (valid ? src : 0) * m.row_vecs;
+        HeadCursor cur(m, lane);
+        for (int base = lane; base < m.row_vecs; base += 32 * UNROLL) {
+            V tmp[UNROLL];
+#pragma unroll
+            for (int u = 0; u < UNROLL; ++u) {
+                const int v = base + u * 32;
+                tmp[u] = (valid && v < m.row_vecs) ? __ldcs(row + v) : z;
+            }
+#pragma unroll
+            for (int u = 0; u < UNROLL; ++u) {
+                if (base + u * 32 < m.row_vecs) __stcs(heads + cur.offset(m, b, s), tmp[u]);
+                cur.advance(m);
+            }
+        }
+    }
+}
+
+template <typename V, int UNROLL>
+__global__ void __launch_bounds__(256) transpose_remove_kernel(const V* __restrict__ heads,
+                                                               const int32_t* __restrict__ cu, HeadMap m,
+                                                               int64_t packed_rows_cap, V* __restrict__ packed) {
+    if (m.batch <= 0) return;
+    int64_t T = __ldg(cu + m.batch);
+    const int64_t cap = (int64_t)m.batch * m.pad_len;
+    if (T > cap) T = cap;
+    if (T > packed_rows_cap) T = packed_rows_cap;
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < T; r += warps) {
+        const int b = owner_of(cu, m.batch, r);
+        const int64_t s = r - __ldg(cu + b);
+        if (s < 0 || s >= m.pad_len) continue;  // offsets inconsistent with pad_len: skip the row
+        V* row = packed + r * m.row_vecs;
+        HeadCursor cur(m, lane);
+        for (int base = lane; base < m.row_vecs; base += 32 * UNROLL) {
+            V tmp[UNROLL];
+#pragma unroll
+            for (int u = 0; u < UNROLL; ++u) {
+                if (base + u * 32 < m.row_vecs) tmp[u] = __ldcs(heads + cur.offset(m, b, (int)s));
+                cur.advance(m);
+            }
+#pragma unroll
+            for (int u = 0; u < UNROLL; ++u) {
+                const int v = base + u * 32;
+                if (v < m.row_vecs) row[v] = tmp[u];
+            }
+        }
+    }
+}
+
+template <typename V>
+static HeadMap head_map(int batch, int pad_len, int parts, int n_heads, int64_t head_bytes) {
+    HeadMap m;
+    m.n_heads = n_heads;
+    m.head_vecs = (int)(head_bytes / (int64_t)sizeof(V));
+    m.row_vecs = parts * n_heads * m.head_vecs;
+    m.batch = batch;
+    m.pad_len = pad_len;
+    m.step_blk = 32 / m.head_vecs;
+    m.step_j = 32 - m.step_blk * m.head_vecs;
+    return m;
+}
+
+cudaError_t launch_transpose_rebuild(const void* packed, const int32_t* cu, int batch, int pad_len, int parts,
+                                     int n_heads, int64_t head_bytes, int64_t packed_rows_cap, void* heads,
+                                     cudaStream_t st) {
+    if (batch <= 0 || pad_len <= 0 || head_bytes == 0) return cudaSuccess;
+    const int grid = row_grid((int64_t)batch * pad_len);
+    const uintptr_t align = reinterpret_cast<uintptr_t>(packed) | reinterpret_cast<uintptr_t>(heads);
+    if (head_bytes % 16 == 0 && align % 16 == 0) {
+        transpose_rebuild_kernel<uint4, 4><<<grid, 256, 0, st>>>(
+            (const uint4*)packed, cu, head_map<uint4>(batch, pad_len, parts, n_heads, head_bytes), packed_rows_cap,
+            (uint4*)heads);
+    } else if (head_bytes % 4 == 0 && align % 4 == 0) {
+        transpose_rebuild_kernel<uint32_t, 8><<<grid, 256, 0, st>>>(
+            (const uint32_t*)packed, cu, head_map<uint32_t>(batch, pad_len, parts, n_heads, head_bytes),
+            packed_rows_cap, (uint32_t*)heads);
+    } else {
+        transpose_rebuild_kernel<uint8_t, 8><<<grid, 256, 0, st>>>(
+            (const uint8_t*)packed, cu, head_map<uint8_t>(batch, pad_len, parts, n_heads, head_bytes),
+            packed_rows_cap, (uint8_t*)heads);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_transpose_remove(const void* heads, const int32_t* cu, int batch, int pad_len, int parts,
+                                    int n_heads, int64_t head_bytes, int64_t packed_rows_cap, void* packed,
+                                    cudaStream_t st) {
+    if (batch <= 0 || head_bytes == 0) return cudaSuccess;
+    const int grid = row_grid((int64_t)batch * pad_len);
+    const uintptr_t align = reinterpret_cast<uintptr_t>(packed) | reinterpret_cast<uintptr_t>(heads);
+    if (head_bytes % 16 == 0 && align % 16 == 0) {
+        transpose_remove_kernel<uint4, 4><<<grid, 256, 0, st>>>(
+            (const uint4*)heads, cu, head_map<uint4>(batch, pad_len, parts, n_heads, head_bytes), packed_rows_cap,
+            (uint4*)packed);
+    } else if (head_bytes % 4 == 0 && align % 4 == 0) {
+        transpose_remove_kernel<uint32_t, 8><<<grid, 256, 0, st>>>(
+            (const uint32_t*)heads, cu, head_map<uint32_t>(batch, pad_len, parts, n_heads, head_bytes),
+            packed_rows_cap, (uint32_t*)packed);
+    } else {
+        transpose_remove_kernel<uint8_t, 8><<<grid, 256, 0, st>>>(
+            (const uint8_t*)heads, cu, head_map<uint8_t>(batch, pad_len, parts, n_heads, head_bytes),
+            packed_rows_cap, (uint8_t*)packed);
+    }
+    return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------ bounded-wait self-test
 
 __global__ void wait_selftest_kernel(int32_t* status, uint64_t timeout_ns) {

@@ -100,8 +100,20 @@ def test_bad_arguments_fail_before_launch(lib):
     with pytest.raises(capi.EnergonError) as e:
         capi.energon_stack_forward(cfg(), [fake], 1, 4096, 8192, 2, 8, 1, 4096, 16384, 20480, 1 << 40, stream=0)
     assert e.value.code == capi.ENERGON_ERR_INVALID_ARGUMENT                # out aliases in
+    for mode in (-1, 3):
+        with pytest.raises(capi.EnergonError) as e:
+            capi.energon_stack_forward(cfg(), [fake], 1, 4096, 8192, 2, 8, mode, 12288, 16384, 20480, 1 << 40,
+                                       stream=0)
+        assert e.value.code == capi.ENERGON_ERR_INVALID_ARGUMENT and "remove_padding" in capi.energon_last_error()
     with pytest.raises(capi.EnergonError):
         capi.energon_selftest_bounded_wait(None, 10, stream=0)
+    for fn in (capi.energon_rce_transpose_padding_rebuild, capi.energon_rce_transpose_padding_remove):
+        for args in ((None, 4096, 2, 8, 3, 2, 64, 2, 8192), (4096, 4096, 2, 8, 0, 2, 64, 2, 8192),
+                     (4096, 4096, 2, 8, 3, 2, 64, 3, 8192), (4096, 4096, 2, -1, 3, 2, 64, 2, 8192),
+                     (4096, 4096, 2, 8, 3, 1 << 16, 1 << 14, 8, 8192)):
+            with pytest.raises(capi.EnergonError) as e:
+                fn(*args, stream=0)
+            assert e.value.code == capi.ENERGON_ERR_INVALID_ARGUMENT
 
 
 def test_binding_rejects_host_tensors(lib):

@@ -174,9 +174,12 @@ def test_stack_packed_equals_padded_and_oracle(oracle_lib, dtype):
     x = synth.normal((B, S, shape.hidden), 12, synth.TID_X, dtype)
     out_pk, st1, hw = stack_run(dtype, shape, L, x, lengths, 12, NONZERO, 1)
     out_pd, st2, _ = stack_run(dtype, shape, L, x, lengths, 12, NONZERO, 0)
-    assert st1 == st2 == 0
-    # the padded run computes pad rows too, yet every valid row must agree bit for bit
+    out_mlp, st6, _ = stack_run(dtype, shape, L, x, lengths, 12, NONZERO, 2)
+    assert st1 == st2 == st6 == 0
+    # the padded run computes pad rows too, yet every valid row must agree bit for bit; so must
+    # the run that packs only around each MLP (attention on the padded rows)
     assert torch.equal(out_pk.view(torch.int16), out_pd.view(torch.int16))
+    assert torch.equal(out_pk.view(torch.int16), out_mlp.view(torch.int16))
     # The stated tolerance is for a layer output.  fp16 meets it through 3 layers; bf16 (unit
     # roundoff 8x fp16's) is held to it over one layer, its 3-layer run to the exact checks.
     L_ref = L if dtype == synth.F16 else 1
@@ -217,8 +220,45 @@ def test_stack_invalid_lengths_and_empty_batch():
     assert (out.view(torch.int16) == 0).all()
     out, st, _ = stack_run(synth.F16, shape, 2, x, np.array([3, -1, 2], np.int32), 4, NONZERO, 0)
     assert st == capi.ENERGON_DEVICE_BAD_LENGTH and (out.view(torch.int16) == 0).all()
-    out, st, _ = stack_run(synth.F16, shape, 2, x, np.zeros(3, np.int32), 4, NONZERO, 1)
-    assert st == 0 and (out.view(torch.int16) == 0).all()
+    out, st, _ = stack_run(synth.F16, shape, 2, x, np.array([3, 17, 2], np.int32), 4, NONZERO, 2)
+    assert st == capi.ENERGON_DEVICE_BAD_LENGTH and (out.view(torch.int16) == 0).all()
+    for mode in (0, 1, 2):
+        out, st, _ = stack_run(synth.F16, shape, 2, x, np.zeros(3, np.int32), 4, NONZERO, mode)
+        assert st == 0 and (out.view(torch.int16) == 0).all()
+
+
+def test_stack_modes_launch_their_own_schedules():
+    """The three modes agree on valid rows by design, so their schedules are told apart by
+    the launch trace: packing once around the stack (1), never (0), or around every MLP (2)."""
+    shape = synth.LayerShape(256, 2, 512)
+    lengths = np.array([5, 16, 9], np.int32)
+    x = synth.normal((3, 16, 256), 3, synth.TID_X, synth.F16)
+    L = 3
+    want = {1: {"remove_padding": 1, "rebuild_padding": 1, "padded_starts": 0},
+            0: {"remove_padding": 0, "rebuild_padding": 1, "padded_starts": 1},
+            2: {"remove_padding": L, "rebuild_padding": L, "padded_starts": 1}}
+    for mode, counts in want.items():
+        capi.energon_trace_start()
+        _, st, _ = stack_run(synth.F16, shape, L, x, lengths, 3, NONZERO, mode)
+        trace = capi.energon_trace_stop()
+        assert st == 0
+        got = {k: trace.get(k, (0, 0.0))[0] for k in counts}
+        assert got == counts, (mode, trace)
+        assert trace["gemm_qkv"][0] == trace["gemm_ffn2"][0] == L
+
+
+@pytest.mark.parametrize("mode", [0, 1, 2])
+def test_stack_without_layers_repacks_input(mode):
+    """Zero layers: every mode returns the valid rows of the input unchanged and zero pads."""
+    shape = synth.LayerShape(256, 2, 512)
+    lengths = np.array([5, 16, 0, 9], np.int32)
+    x = synth.normal((4, 16, 256), 8, synth.TID_X, synth.F16)
+    out, st, _ = stack_run(synth.F16, shape, 0, x, lengths, 8, NONZERO, mode)
+    assert st == 0
+    got = out.cpu().view(torch.int16).numpy()
+    for b in range(4):
+        assert np.array_equal(got[b, :lengths[b]], x[b, :lengths[b]].view(np.int16))
+        assert not got[b, lengths[b]:].any()
 
 
 def test_bounded_wait_times_out_and_context_survives():

@@ -7,8 +7,9 @@
   outputs.  Causal attention makes the first p outputs of a sequence a function of its
   first p tokens only, so the oracle computes them exactly from a p-token prefix: whole
   short sequences and the first positions of long ones.  Properties that hold at any size
-  are checked on the full output: pad rows are zero, the padded path gives the same valid
-  rows bit for bit, and different garbage in the pad positions changes no valid row.
+  are checked on the full output: pad rows are zero, the padded path and the path that
+  packs only around each MLP give the same valid rows bit for bit, and different garbage
+  in the pad positions changes no valid row.
 """
 import numpy as np
 import pytest
@@ -84,6 +85,9 @@ def full_size_case(wl, oracle_lib, sample_plan):
     out_pad = run_stack(wl, dev_layers, x, lengths, S, 0)         # padded path: same valid rows
     assert torch.equal(out.view(torch.int16), out_pad.view(torch.int16))
     del out_pad
+    out_mlp = run_stack(wl, dev_layers, x, lengths, S, 2)         # packing around each MLP only
+    assert torch.equal(out.view(torch.int16), out_mlp.view(torch.int16))
+    del out_mlp
     x2 = wl.x_padded(synth.TID_X_ALT_PADS)                        # other pad garbage: same rows
     for b in range(wl.batch):
         x2[b, :lengths[b]] = x[b, :lengths[b]]
