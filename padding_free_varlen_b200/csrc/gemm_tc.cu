@@ -193,6 +193,136 @@ __device__ __forceinline__ void drain_256(uint32_t tbase, const TcParams& p, int
     }
 }
 
+// Staging buffer of one epilogue warp: 32 rows x 32 columns of 16-bit values,
+// 64 bytes per row, in the TMA 64-byte swizzle (the 16-byte chunk index is XORed
+// with bits 1-2 of the row), so that 32 threads each touching their own row hit
+// every bank once per 128 bytes.
+__device__ __forceinline__ uint32_t stage_off(int row, int chunk) {
+    return (uint32_t)(row * 64 + ((chunk ^ ((row >> 1) & 3)) << 4));
+}
+
+// One warp drains 256 accumulator columns of its 32 rows through shared memory:
+// per 32-column chunk, TMEM -> registers -> bias / GELU / residual -> one
+// rounding -> the warp's staging buffer -> one TMA store of the 32 x 32 box.
+// The residual box of the next chunk is fetched by TMA into the other buffer
+// while the current one is processed.  The accumulator is handed back (arrival
+// on `tempty_cluster`) as soon as its last columns are in registers.  Every row
+// of the warp must be valid (rows < M); the warp holding the last valid row
+// takes drain_256 instead.  Returns false if a residual copy timed out.
+template <typename T, int EPI>
+__device__ __forceinline__ bool drain_256_staged(uint32_t tbase, const TcParams& p, const CUtensorMap* tmO,
+                                                 const CUtensorMap* tmR, uint8_t* sbuf, uint64_t* rbar,
+                                                 uint32_t& rpar, int row_base, int col_base, uint32_t tempty_cluster,
+                                                 const volatile int* abort_flag) {
+    const int lane = threadIdx.x & 31;
+    uint32_t r[2][32];
+    bool ok = true;
+    uint32_t pend = 0;  // buffers with a residual copy in flight
+    if (lane == 0) {
+        bulk_wait_read<0>();  // the previous tile's stores no longer read either buffer
+        if (EPI == EPI_BIAS_RESIDUAL) {
+            mbar_arrive_expect_tx(&rbar[0], 32 * 64);
+            tma_load_2d(sbuf, tmR, &rbar[0], col_base, row_base);
+        }
+    }
+    if (EPI == EPI_BIAS_RESIDUAL) pend = 1u;
+    __syncwarp();
+    tmem_ld_x16(tbase, r[0]);
+    tmem_ld_x16(tbase + 16, r[0] + 16);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        const int cur = c & 1;
+        uint8_t* buf = sbuf + cur * 2048;
+        tmem_wait_ld_regs(r[cur]);
+        if (c + 1 < 8) {
+            tmem_ld_x16(tbase + (c + 1) * 32, r[cur ^ 1]);
+            tmem_ld_x16(tbase + (c + 1) * 32 + 16, r[cur ^ 1] + 16);
+        } else {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(tempty_cluster);
+        }
+        const int col0 = col_base + c * 32;
+        if (EPI == EPI_BIAS_RESIDUAL && c + 1 < 8) {
+            if (lane == 0) {
+                bulk_wait_read<0>();  // chunk c-1's store has read the other buffer
+                mbar_arrive_expect_tx(&rbar[cur ^ 1], 32 * 64);
+                tma_load_2d(sbuf + (cur ^ 1) * 2048, tmR, &rbar[cur ^ 1], col0 + 32, row_base);
+            }
+            pend |= 1u << (cur ^ 1);
+        }
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[cur][j]);
+        if (p.bias != nullptr) {
+            const uint4* bp = reinterpret_cast<const uint4*>(static_cast<const T*>(p.bias) + col0);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const uint4 w = __ldg(bp + q);
+                const uint32_t* ww = reinterpret_cast<const uint32_t*>(&w);
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const float2 f = unpack2<T>(ww[h]);
+                    v[q * 8 + 2 * h] += f.x;
+                    v[q * 8 + 2 * h + 1] += f.y;
+                }
+            }
+        }
+        if (EPI == EPI_BIAS_GELU) {
+            if (p.gelu_tanh) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] = gelu_tanh_fast(v[j]);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] = gelu_f(v[j], false);
+            }
+        }
+        if (EPI == EPI_BIAS_RESIDUAL) {
+            const bool got = mbar_wait_bounded(&rbar[cur], (rpar >> cur) & 1u, abort_flag, p.timeout_ns);
+            if (!__all_sync(0xffffffffu, got)) {
+                // copies still in flight get one more bounded wait before the warp gives up
+                if (lane == 0)
+                    for (int b = 0; b < 2; ++b)
+                        if (pend & (1u << b)) mbar_wait_bounded(&rbar[b], (rpar >> b) & 1u, nullptr, p.timeout_ns);
+                ok = false;
+                break;
+            }
+            rpar ^= 1u << cur;
+            pend &= ~(1u << cur);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const uint4 w = *reinterpret_cast<const uint4*>(buf + stage_off(lane, q));
+                const uint32_t* ww = reinterpret_cast<const uint32_t*>(&w);
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const float2 f = unpack2<T>(ww[h]);
+                    v[q * 8 + 2 * h] += f.x;
+                    v[q * 8 + 2 * h + 1] += f.y;
+                }
+            }
+        } else if (c >= 2) {
+            if (lane == 0) bulk_wait_read<1>();  // chunk c-2's store has read this buffer
+            __syncwarp();
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            uint4 o;
+            o.x = pack2<T>(v[q * 8 + 0], v[q * 8 + 1]);
+            o.y = pack2<T>(v[q * 8 + 2], v[q * 8 + 3]);
+            o.z = pack2<T>(v[q * 8 + 4], v[q * 8 + 5]);
+            o.w = pack2<T>(v[q * 8 + 6], v[q * 8 + 7]);
+            *reinterpret_cast<uint4*>(buf + stage_off(lane, q)) = o;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_2d(tmO, buf, col0, row_base);
+            bulk_commit();
+        }
+    }
+    return ok;
+}
+
 // One warp writes its 32 rows x 256 accumulator columns as fp32 partial sums.
 __device__ __forceinline__ void drain_256_partial(uint32_t tbase, float* part, int N, int row, int col_base, int M) {
 #pragma unroll 1
@@ -463,24 +593,29 @@ struct PairCfg {
     static constexpr int SLOT_COLS = MT * PBN;
     static constexpr int EPI_WARPS = 4 * MT;
     static constexpr int THREADS = 128 + 32 * EPI_WARPS;
-    static constexpr int SMEM = STAGES * STAGE + 1024 + 256;
+    static constexpr int EPI_STAGE = 4096;  // per epilogue warp: two 32 x 32 staging buffers
+    static constexpr int SMEM = STAGES * STAGE + EPI_WARPS * EPI_STAGE + 1024 + 384;
 };
 
 template <typename T, int EPI, int MT>
 __global__ void __launch_bounds__(PairCfg<MT>::THREADS, 1)
-    gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const TcParams p) {
+    gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmR,
+                    const TcParams p) {
     using C = PairCfg<MT>;
     constexpr int NST = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = base;                    // [stage][MT][128 rows x 128 B]
     uint8_t* sB = base + NST * C::A_STAGE;  // [stage][128 rows x 128 B]
-    uint64_t* full = reinterpret_cast<uint64_t*>(sB + NST * PB_STAGE);
+    uint8_t* sE = sB + NST * PB_STAGE;      // [epilogue warp][2][32 rows x 64 B]
+    uint64_t* full = reinterpret_cast<uint64_t*>(sE + C::EPI_WARPS * C::EPI_STAGE);
     uint64_t* empty = full + NST;
     uint64_t* tfull = empty + NST;
     uint64_t* tempty = tfull + 2;
     uint64_t* drain = tempty + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    uint64_t* rbar = drain + 1;             // [epilogue warp][2] residual copies
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rbar + 2 * C::EPI_WARPS);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -495,7 +630,17 @@ __global__ void __launch_bounds__(PairCfg<MT>::THREADS, 1)
     const int num_mt = (num_m + MT - 1) / MT;            // pair tiles along M
     const int num_n = (p.N + PBN - 1) / PBN;
     const int total = num_mt * num_n;
-    if (pair >= total) return;
+    // Wave tail: when the last round of pair tiles would leave more than half of the pairs
+    // idle, its tiles are issued as two half units of one row tile each, so the round takes
+    // half as long.  A row's arithmetic is the same in a half unit (the same MMA per row
+    // tile, the same K order), so results do not depend on how the tiles were cut.
+    int full_units = total, split_tiles = 0;
+    if (MT == 2 && total > npairs) {
+        const int rem = total % npairs;
+        if (rem != 0 && 2 * rem <= npairs) full_units = total - rem, split_tiles = rem;
+    }
+    const int units = full_units + 2 * split_tiles;
+    if (pair >= units) return;
     const int num_kb = (p.K + PBK - 1) / PBK;
     // Tile order: groups of 8 row tiles (2048 rows); inside a group every row tile of a
     // column runs before the next column, so each weight panel is fetched about once per
@@ -503,6 +648,15 @@ __global__ void __launch_bounds__(PairCfg<MT>::THREADS, 1)
     // on the four GPT-3 shapes it is within 1 % of every other order tried and ahead of
     // the rest; L2 eviction-priority hints made it 10 % slower.
     const int group = 8 / MT;
+    // unit u -> pair tile t and its row tiles [i0, i1)
+    auto unit_of = [&](int u, int& t, int& i0, int& i1) {
+        if (u < full_units) {
+            t = u, i0 = 0, i1 = MT;
+        } else {
+            const int v = u - full_units;
+            t = full_units + (v >> 1), i0 = v & 1, i1 = i0 + 1;
+        }
+    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < NST; ++s) {
@@ -514,12 +668,15 @@ __global__ void __launch_bounds__(PairCfg<MT>::THREADS, 1)
             mbar_init(&tempty[a], 2 * C::EPI_WARPS);  // every epilogue warp of both CTAs
         }
         mbar_init(drain, 1);
+        for (int w = 0; w < 2 * C::EPI_WARPS; ++w) mbar_init(&rbar[w], 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmO);
+        if (EPI == EPI_BIAS_RESIDUAL) tma_prefetch_desc(&tmR);
     }
     if (warp == 2) {
         tmem_alloc_pair(tmem_slot, TMEM_COLS);
@@ -535,9 +692,11 @@ __global__ void __launch_bounds__(PairCfg<MT>::THREADS, 1)
         int stage = 0;
         uint32_t phase = 0, pend_mask = 0, pend_par = 0;
         bool ok = true;
-        for (int t = pair; t < total && ok; t += npairs) {
-            int mt, n;
+        for (int u = pair; u < units && ok; u += npairs) {
+            int t, i0, i1, mt, n;
+            unit_of(u, t, i0, i1);
             tile_coords(t, num_mt, num_n, group, 0, mt, n);
+            const uint32_t tx = 2u * (uint32_t)((i1 - i0) * PA_STAGE + PB_STAGE);
             for (int kb = 0; kb < num_kb; ++kb) {
                 if (!warp_wait<true>(&empty[stage], phase ^ 1u, abort_flag, p.timeout_ns)) {
                     ok = false;
@@ -545,11 +704,12 @@ __global__ void __launch_bounds__(PairCfg<MT>::THREADS, 1)
                 }
                 if (lane == 0) {
                     const uint32_t bar0 = mapa_shared(smem_u32(&full[stage]), 0);
-                    if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE);
+                    if (leader) mbar_arrive_expect_tx(&full[stage], tx);
 #pragma unroll
                     for (int i = 0; i < MT; ++i)
-                        tma_load_2d_pair(sA + stage * C::A_STAGE + i * PA_STAGE, &tmA, bar0, kb * PBK,
-                                         (mt * MT + i) * PBM + (int)rank * 128);
+                        if (i >= i0 && i < i1)
+                            tma_load_2d_pair(sA + stage * C::A_STAGE + i * PA_STAGE, &tmA, bar0, kb * PBK,
+                                             (mt * MT + i) * PBM + (int)rank * 128);
                     tma_load_2d_pair(sB + stage * PB_STAGE, &tmB, bar0, kb * PBK, n * PBN + (int)rank * 128);
                 }
                 pend_mask |= 1u << stage;
@@ -579,7 +739,9 @@ __global__ void __launch_bounds__(PairCfg<MT>::THREADS, 1)
         int stage = 0, local = 0;
         uint32_t phase = 0;
         bool ok = true;
-        for (int t = pair; t < total && ok; t += npairs, ++local) {
+        for (int u = pair; u < units && ok; u += npairs, ++local) {
+            int t, i0, i1;
+            unit_of(u, t, i0, i1);
             const int slot = local % C::SLOTS;
             const uint32_t use = (uint32_t)(local / C::SLOTS) & 1u;
             if (!warp_wait<true>(&tempty[slot], use ^ 1u, abort_flag, p.timeout_ns)) {
@@ -596,14 +758,25 @@ __global__ void __launch_bounds__(PairCfg<MT>::THREADS, 1)
                 tc_fence_after();
                 if (lane == 0) {
                     const uint64_t b0 = smem_desc_k128(smem_u32(sB + stage * PB_STAGE));
+                    // One thread issues an MMA every ~128 tensor cycles here, so the issue
+                    // loops stay fully unrolled (a runtime-bounded loop measured 11 % slower).
+                    if (i1 - i0 == MT) {
 #pragma unroll
-                    for (int k = 0; k < PBK / 16; ++k) {
+                        for (int k = 0; k < PBK / 16; ++k) {
 #pragma unroll
-                        for (int i = 0; i < MT; ++i) {
-                            const uint64_t a0 = smem_desc_k128(smem_u32(sA + stage * C::A_STAGE + i * PA_STAGE));
-                            umma_f16_pair(d_tmem + (uint32_t)(i * PBN), a0 + 2 * k, b0 + 2 * k, idesc,
-                                          (kb | k) != 0 ? 1u : 0u);
+                            for (int i = 0; i < MT; ++i) {
+                                const uint64_t a0 =
+                                    smem_desc_k128(smem_u32(sA + stage * C::A_STAGE + i * PA_STAGE));
+                                umma_f16_pair(d_tmem + (uint32_t)(i * PBN), a0 + 2 * k, b0 + 2 * k, idesc,
+                                              (kb | k) != 0 ? 1u : 0u);
+                            }
                         }
+                    } else {
+                        const uint64_t a0 = smem_desc_k128(smem_u32(sA + stage * C::A_STAGE + i0 * PA_STAGE));
+                        const uint32_t dt = d_tmem + (uint32_t)(i0 * PBN);
+#pragma unroll
+                        for (int k = 0; k < PBK / 16; ++k)
+                            umma_f16_pair(dt, a0 + 2 * k, b0 + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
                     }
                     umma_commit_pair(&empty[stage], 0x3);
                 }
@@ -627,9 +800,14 @@ __global__ void __launch_bounds__(PairCfg<MT>::THREADS, 1)
         // ---------------------------------------------------------------- epilogue (both CTAs)
         const int q = warp & 3;             // TMEM lane quarter this warp may access
         const int i = (warp - 4) >> 2;      // row tile of the pair tile this warp drains
+        uint8_t* sbuf = sE + (warp - 4) * C::EPI_STAGE;
+        uint64_t* rb = rbar + 2 * (warp - 4);
+        uint32_t rpar = 0;
         int local = 0;
         bool ok = true;
-        for (int t = pair; t < total; t += npairs, ++local) {
+        for (int u = pair; u < units; u += npairs, ++local) {
+            int t, i0, i1;
+            unit_of(u, t, i0, i1);
             const int slot = local % C::SLOTS;
             const uint32_t use = (uint32_t)(local / C::SLOTS) & 1u;
             if (!warp_wait(&tfull[slot], use, abort_flag, p.timeout_ns)) {
@@ -637,20 +815,37 @@ __global__ void __launch_bounds__(PairCfg<MT>::THREADS, 1)
                 break;
             }
             tc_fence_after();
-            int mt, n;
-            tile_coords(t, num_mt, num_n, group, 0, mt, n);
-            const int row = (mt * MT + i) * PBM + (int)rank * 128 + q * 32 + lane;
-            const uint32_t tbase =
-                tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(slot * C::SLOT_COLS + i * PBN);
-            drain_256<T, EPI>(tbase, p, row, n * PBN, M);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[slot]), 0));
+            const uint32_t tempty_cluster = mapa_shared(smem_u32(&tempty[slot]), 0);
+            bool handed_back = false;
+            if (i >= i0 && i < i1) {  // a half unit leaves the other row tile's warps idle
+                int mt, n;
+                tile_coords(t, num_mt, num_n, group, 0, mt, n);
+                const int row_base = (mt * MT + i) * PBM + (int)rank * 128 + q * 32;
+                const uint32_t tbase =
+                    tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(slot * C::SLOT_COLS + i * PBN);
+                if (row_base + 32 <= M) {
+                    ok = drain_256_staged<T, EPI>(tbase, p, &tmO, &tmR, sbuf, rb, rpar, row_base, n * PBN,
+                                                  tempty_cluster, abort_flag);
+                    handed_back = ok;
+                } else {
+                    drain_256<T, EPI>(tbase, p, row_base + lane, n * PBN, M);
+                }
+            }
+            if (!ok) break;
+            if (!handed_back) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(tempty_cluster);
+            }
         }
-        if (!ok && lane == 0) {
-            *abort_flag = 1;
-            status_or(p.status, ENERGON_DEVICE_TIMEOUT);
+        if (lane == 0) {
+            if (!ok) {
+                *abort_flag = 1;
+                status_or(p.status, ENERGON_DEVICE_TIMEOUT);
+            }
+            bulk_wait<0>();  // every output store has landed before the CTA retires
         }
+        __syncwarp();
     }
     tc_fence_before();
     cluster_sync();  // neither CTA leaves while its pair may still read or signal its shared memory
@@ -687,6 +882,20 @@ static CUresult make_tmap(CUtensorMap* m, int dtype, const void* ptr, int64_t K,
               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
+// 2-D row-major tensor [rows, N] of 16-bit elements, box 32 x 32, 64-byte swizzle.
+static CUresult make_tmap_io(CUtensorMap* m, int dtype, const void* ptr, int64_t N, int64_t rows) {
+    auto fn = encode_fn();
+    if (!fn) return CUDA_ERROR_NOT_FOUND;
+    const CUtensorMapDataType dt =
+        dtype == ENERGON_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)N * 2};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
 bool gemm_tc_supported(const GemmArgs& a) {
     if (a.dtype != ENERGON_F16 && a.dtype != ENERGON_BF16) return false;
     if (a.K < TBK || a.K % TBK != 0 || a.N < TBN || a.N % TBN != 0) return false;
@@ -713,8 +922,8 @@ static cudaError_t tc_launch(const CUtensorMap& ta, const CUtensorMap& tb, const
 }
 
 template <typename T, int EPI, int MT>
-static cudaError_t tc2_launch(const CUtensorMap& ta, const CUtensorMap& tb, const TcParams& p, int pairs,
-                              cudaStream_t st) {
+static cudaError_t tc2_launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to,
+                              const CUtensorMap& tr, const TcParams& p, int pairs, cudaStream_t st) {
     using C = PairCfg<MT>;
     static int max_pairs = -1;
     cudaLaunchAttribute attr[1];
@@ -747,16 +956,16 @@ static cudaError_t tc2_launch(const CUtensorMap& ta, const CUtensorMap& tb, cons
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<T, EPI, MT>, ta, tb, p);
+    return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<T, EPI, MT>, ta, tb, to, tr, p);
 }
 
 template <typename T, int MT>
-static cudaError_t tc2_dispatch(int epi, const CUtensorMap& ta, const CUtensorMap& tb, const TcParams& p, int pairs,
-                                cudaStream_t st) {
+static cudaError_t tc2_dispatch(int epi, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to,
+                                const CUtensorMap& tr, const TcParams& p, int pairs, cudaStream_t st) {
     switch (epi) {
-    case EPI_BIAS: return tc2_launch<T, EPI_BIAS, MT>(ta, tb, p, pairs, st);
-    case EPI_BIAS_GELU: return tc2_launch<T, EPI_BIAS_GELU, MT>(ta, tb, p, pairs, st);
-    default: return tc2_launch<T, EPI_BIAS_RESIDUAL, MT>(ta, tb, p, pairs, st);
+    case EPI_BIAS: return tc2_launch<T, EPI_BIAS, MT>(ta, tb, to, tr, p, pairs, st);
+    case EPI_BIAS_GELU: return tc2_launch<T, EPI_BIAS_GELU, MT>(ta, tb, to, tr, p, pairs, st);
+    default: return tc2_launch<T, EPI_BIAS_RESIDUAL, MT>(ta, tb, to, tr, p, pairs, st);
     }
 }
 
@@ -796,11 +1005,22 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st, char* err, size_t
         p.group_m = 1;
         const int64_t tiles_cap = (int64_t)num_m_cap * num_n;
         const int pairs = (int)(tiles_cap < device_sm_count() / 2 ? tiles_cap : device_sm_count() / 2);
+        // Output (and residual) as 32 x 32 boxes, 64-byte swizzle: the epilogue's staged
+        // stores and residual loads.  Only boxes of rows below the live row count are
+        // ever copied, so the maps may span the whole buffer capacity.
+        CUtensorMap to, tr;
+        CUresult r3 = make_tmap_io(&to, a.dtype, a.out, a.N, a.M_cap);
+        CUresult r4 = a.epilogue == EPI_BIAS_RESIDUAL ? make_tmap_io(&tr, a.dtype, a.residual, a.N, a.M_cap) : r3;
+        if (a.epilogue != EPI_BIAS_RESIDUAL) tr = to;
+        if (r3 != CUDA_SUCCESS || r4 != CUDA_SUCCESS) {
+            if (err) snprintf(err, errlen, "cuTensorMapEncodeTiled failed (out: %d, residual: %d)", (int)r3, (int)r4);
+            return cudaErrorInvalidValue;
+        }
         if (mt == 2)
-            return bf ? tc2_dispatch<__nv_bfloat16, 2>(a.epilogue, ta, tb, p, pairs, st)
-                      : tc2_dispatch<__half, 2>(a.epilogue, ta, tb, p, pairs, st);
-        return bf ? tc2_dispatch<__nv_bfloat16, 1>(a.epilogue, ta, tb, p, pairs, st)
-                  : tc2_dispatch<__half, 1>(a.epilogue, ta, tb, p, pairs, st);
+            return bf ? tc2_dispatch<__nv_bfloat16, 2>(a.epilogue, ta, tb, to, tr, p, pairs, st)
+                      : tc2_dispatch<__half, 2>(a.epilogue, ta, tb, to, tr, p, pairs, st);
+        return bf ? tc2_dispatch<__nv_bfloat16, 1>(a.epilogue, ta, tb, to, tr, p, pairs, st)
+                  : tc2_dispatch<__half, 1>(a.epilogue, ta, tb, to, tr, p, pairs, st);
     }
     const int num_m_cap = (a.M_cap + TBM - 1) / TBM, num_n = a.N / TBN;
     // Rows of A kept hot per raster group: about 48 MiB of the 126 MB L2.

@@ -212,6 +212,29 @@ def test_stack_packed_equals_padded_and_oracle(oracle_lib, dtype):
                              f"alone vs batch seq {b}")
 
 
+def test_gemm_wave_tail_cut_does_not_change_rows(oracle_lib):
+    """Hidden 1024, FFN 2560, 4096 valid tokens in a 16 x 512 batch.  On 148 SMs (74 CTA
+    pairs) the packed QKV and FFN1 GEMMs have 96 and 80 pair tiles, so their last round is
+    issued as half tiles; the padded run's 192 and 160 tiles are cut differently (not at
+    all, and 12 tiles).  Valid rows must agree bit for bit across the three modes, and
+    match the oracle."""
+    shape = synth.LayerShape(1024, 8, 2560)
+    B, S = 16, 512
+    lengths = np.array([192, 320] * 8, np.int32)
+    x = synth.normal((B, S, shape.hidden), 31, synth.TID_X, synth.F16)
+    out1, st1, hw = stack_run(synth.F16, shape, 1, x, lengths, 31, NONZERO, 1)
+    out0, st0, _ = stack_run(synth.F16, shape, 1, x, lengths, 31, NONZERO, 0)
+    out2, st2, _ = stack_run(synth.F16, shape, 1, x, lengths, 31, NONZERO, 2)
+    assert st0 == st1 == st2 == 0
+    assert torch.equal(out1.view(torch.int16), out0.view(torch.int16))
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+    sel = [0, 1]
+    ref = oracle_lib.layer_padded(synth.to_f64(x[sel], synth.F16), lengths[sel], hw[0], shape.n_heads)
+    for j, b in enumerate(sel):
+        n = int(lengths[b])
+        check_end_to_end(to_f64(out1[b, :n]), ref[j, :n], synth.F16, f"wave-tail layer seq {b}")
+
+
 def test_stack_invalid_lengths_and_empty_batch():
     shape = synth.LayerShape(256, 2, 512)
     x = synth.normal((3, 16, 256), 4, synth.TID_X, synth.F16)
