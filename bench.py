@@ -343,7 +343,7 @@ def run_energon(args, dist: Dist):
 
     # ---- roofline of the dominant kernel (the tcgen05 GEMM, four shapes per layer)
     peaks = load_peaks()
-    gemm_names = ("gemm_qkv", "gemm_out_proj", "gemm_ffn1", "gemm_ffn2")
+    gemm_names = ("gemm_qkv", "gemm_out_proj", "gemm_ffn1", "gemm_ffn2", "gemm_ffn2_rebuild")
     g_launch = sum(trace.get(n, (0, 0.0))[0] for n in gemm_names)
     g_ms = sum(trace.get(n, (0, 0.0))[1] for n in gemm_names)
     flops_per_token_layer = 24 * H * H            # 2*(3H*H + H*H + 4H*H + 4H*H)
@@ -359,14 +359,17 @@ def run_energon(args, dist: Dist):
                              f"burst {peaks['tflops']}",
                 "traffic": traffic, "algorithmic_flops_per_launch": gemm_flops_per_launch,
                 "ms_per_launch": g_ms / max(1, g_launch)}
-    # memory-bound companions measured in the same region
+    # memory-bound companions measured in the same region: the packing fused into the first
+    # LayerNorm (reads the padded rows once, writes the packed rows and their normalisation)
+    # and the pad zeroing; standalone remove / rebuild are timed after the main region
     aux = {}
     e = 2 if tdt != torch.float32 else 4
-    for name, nbytes in (("remove_padding", 2 * T * H * e), ("rebuild_padding", T * H * e + B * S * H * e)):
+    for name, nbytes, per in (("layernorm_remove", 3 * T * H * e, 1), ("zero_pads", (B * S - T) * H * e, 1)):
         if name in trace and trace[name][1] > 0:
             gbs = nbytes * trace[name][0] / (trace[name][1] / 1e3) / 1e9
             aux[name] = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": gbs / peaks["hbm_gbs"], "algorithmic_bytes_per_launch": nbytes}
+                         "frac": gbs / peaks["hbm_gbs"], "algorithmic_bytes_per_launch": nbytes,
+                         "ms_per_launch": trace[name][1] / trace[name][0]}
 
     # ---- end to end through the C ABI with host buffers (H2D + stack + D2H every step)
     e2e = None
@@ -430,6 +433,26 @@ def run_energon(args, dist: Dist):
         del qkv_rows, heads, back
         if int(st.item()) != 0:
             raise RuntimeError(f"device status {int(st.item())} after the transpose forms")
+
+    # ---- the standalone packing operators on this workload (energon_rce_remove_padding /
+    # energon_rce_rebuild_padding), CUDA events on the launching stream
+    if not args.no_transpose:
+        cu_sa = torch.empty(B + 1, dtype=torch.int32, device=dev)
+        capi.energon_rce_offsets(d_len, B, S, cu_sa, st, stream)
+        pk = torch.empty((B * S, H), dtype=tdt, device=dev)
+        ks = max(3, args.steps)
+        for name, fn, nbytes in (
+                ("remove_padding", lambda: capi.energon_rce_remove_padding(d_in, cu_sa, B, S, H, e, pk, stream),
+                 2 * T * H * e),
+                ("rebuild_padding", lambda: capi.energon_rce_rebuild_padding(pk, cu_sa, B, S, H, e, d_out, stream),
+                 T * H * e + B * S * H * e)):
+            fn()
+            ms_t = timed(fn, ks) / ks
+            gbs = nbytes / (ms_t / 1e3) / 1e9
+            aux[name] = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "algorithmic_bytes_per_launch": nbytes,
+                         "ms_per_launch": ms_t, "standalone": True}
+        del pk
 
     launches = sum(v[0] for v in trace.values())
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": dist.world, "steps": args.steps,

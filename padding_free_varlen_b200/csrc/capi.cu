@@ -210,16 +210,33 @@ GemmArgs gemm_base(const energon_layer_config& c, const int32_t* cu, int batch, 
 
 // Attention sub-layer on the rows described by cu (row starts; rows valid = cu[batch]):
 //   x1 = x + attention(LN1(x) W_qkv^T + b_qkv) W_o^T + b_o
+// With `padded` set, x is gathered from that [batch, max_len, H] tensor by the first
+// LayerNorm (transpose_padding_remove fused into it), which also writes the packed
+// rows to x (then the residual stream's buffer).
 int attention_sublayer(const energon_layer_config& c, const energon_layer_weights& w, const void* x,
                        const int32_t* cu, int batch, int max_len, void* x1, int32_t* status, const LayerWs& ws,
-                       cudaStream_t st) {
+                       cudaStream_t st, const void* padded = nullptr) {
     const int H = c.hidden;
     const int M_cap = batch * max_len;
     const int A_rows = (int)rows_alloc(batch, max_len);
     const int32_t* d_rows = cu + batch;
-    CK(traced("layernorm", st,
-              [&] { return launch_layernorm(c.dtype, x, w.ln1_g, w.ln1_b, ws.a, d_rows, M_cap, H, c.ln_eps, status, st); }),
-       "ln1");
+    if (padded != nullptr) {
+        LnGather gth;
+        gth.cu = cu, gth.batch = batch, gth.pad_len = max_len, gth.copy = const_cast<void*>(x);
+        CK(traced("layernorm_remove", st,
+                  [&] {
+                      return launch_layernorm(c.dtype, padded, w.ln1_g, w.ln1_b, ws.a, d_rows, M_cap, H, c.ln_eps,
+                                              status, st, gth);
+                  }),
+           "ln1 + remove");
+    } else {
+        CK(traced("layernorm", st,
+                  [&] {
+                      return launch_layernorm(c.dtype, x, w.ln1_g, w.ln1_b, ws.a, d_rows, M_cap, H, c.ln_eps, status,
+                                              st);
+                  }),
+           "ln1");
+    }
     GemmArgs g = gemm_base(c, cu, batch, max_len, status, ws);
     g.A = ws.a, g.W = w.w_qkv, g.bias = w.b_qkv, g.residual = nullptr, g.out = ws.qkv;
     g.N = 3 * H, g.K = H, g.epilogue = EPI_BIAS;
@@ -236,8 +253,12 @@ int attention_sublayer(const energon_layer_config& c, const energon_layer_weight
 }
 
 // MLP sub-layer: y = x1 + GELU(LN2(x1) W_1^T + b_1) W_2^T + b_2 (y may alias nothing but itself).
+// With `padded_out` set and the FFN2 GEMM on the CTA-pair kernel, its epilogue stores each
+// row at its padded position in padded_out (transpose_padding_rebuild fused into it; pad
+// rows are left alone) and *scattered is set; otherwise the rows go to y.
 int mlp_sublayer(const energon_layer_config& c, const energon_layer_weights& w, const void* x1, const int32_t* cu,
-                 int batch, int max_len, void* y, int32_t* status, const LayerWs& ws, cudaStream_t st) {
+                 int batch, int max_len, void* y, int32_t* status, const LayerWs& ws, cudaStream_t st,
+                 void* padded_out = nullptr, bool* scattered = nullptr) {
     const int H = c.hidden, F = c.ffn;
     const int M_cap = batch * max_len;
     const int32_t* d_rows = cu + batch;
@@ -250,6 +271,16 @@ int mlp_sublayer(const energon_layer_config& c, const energon_layer_weights& w, 
     if (int r = run_gemm(g, st, "gemm_ffn1")) return r;
     g.A = ws.f, g.W = w.w_2, g.bias = w.b_2, g.residual = x1, g.out = y;
     g.N = H, g.K = F, g.epilogue = EPI_BIAS_RESIDUAL;
+    if (scattered) *scattered = false;
+    if (padded_out != nullptr) {
+        GemmArgs gs = g;
+        gs.out = padded_out;
+        gs.scatter_cu = cu, gs.scatter_batch = batch, gs.scatter_pad_len = max_len;
+        if (gemm_tc_scatter_ok(gs)) {
+            if (scattered) *scattered = true;
+            return run_gemm(gs, st, "gemm_ffn2_rebuild");
+        }
+    }
     return run_gemm(g, st, "gemm_ffn2");
 }
 
@@ -397,16 +428,36 @@ int energon_stack_forward(const energon_layer_config* cfg, const energon_layer_w
 
     CK(traced("offsets", st, [&] { return launch_offsets(lengths, batch, pad_len, ws.cu, d_status, st); }),
        "offsets");
-    if (remove_padding == 1) {
+    if (remove_padding == 1 && n_layers == 0) {
         CK(traced("remove_padding", st,
                   [&] { return launch_remove(padded_in, ws.cu, batch, pad_len, row_bytes, ws.x, R, d_status, st); }),
            "remove");
-        for (int l = 0; l < n_layers; ++l)
-            if (int r = layer_impl(*cfg, layers[l], ws.x, ws.cu, batch, pad_len, ws.x, d_status, ws.layer, st))
-                return r;
         CK(traced("rebuild_padding", st,
                   [&] { return launch_rebuild(ws.x, ws.cu, ws.cu, batch, pad_len, row_bytes, R, padded_out, st); }),
            "rebuild");
+    } else if (remove_padding == 1) {
+        // The packing is fused into the first LayerNorm (it gathers the valid rows of
+        // padded_in and writes them to the residual stream ws.x) and the scatter back into
+        // the last FFN2 GEMM's epilogue (each row stored at its padded position); the pad
+        // rows of padded_out are zeroed up front.
+        CK(traced("zero_pads", st, [&] { return launch_zero_pads(ws.cu, batch, pad_len, row_bytes, padded_out, st); }),
+           "zero pads");
+        bool scattered = false;
+        for (int l = 0; l < n_layers; ++l) {
+            const energon_layer_weights& w = layers[l];
+            if (int r = attention_sublayer(*cfg, w, ws.x, ws.cu, batch, pad_len, ws.layer.x1, d_status, ws.layer, st,
+                                           l == 0 ? padded_in : nullptr))
+                return r;
+            if (int r = mlp_sublayer(*cfg, w, ws.layer.x1, ws.cu, batch, pad_len, ws.x, d_status, ws.layer, st,
+                                     l + 1 == n_layers ? padded_out : nullptr, &scattered))
+                return r;
+        }
+        if (!scattered)
+            CK(traced("rebuild_padding", st,
+                      [&] {
+                          return launch_rebuild(ws.x, ws.cu, ws.cu, batch, pad_len, row_bytes, R, padded_out, st);
+                      }),
+               "rebuild");
     } else if (remove_padding == 2) {
         // Elimination for the MLP only, as the QbitAI article's "Runtime" section states it:
         // each layer's attention sub-layer runs on all batch * pad_len rows; its output is

@@ -181,6 +181,17 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
         : "memory");
 }
 
+// Largest b in [0, batch) with cu[b] <= r: the sequence that owns packed row r.
+__device__ __forceinline__ int owner_of(const int32_t* __restrict__ cu, int batch, int64_t r) {
+    int lo = 0, hi = batch - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (__ldg(cu + mid) <= r) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
 // 2-D tile store from this CTA's shared memory (bulk-group completion).
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, const void* smem_src, int c0, int c1) {
     asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(

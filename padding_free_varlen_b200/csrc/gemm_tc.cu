@@ -61,7 +61,18 @@ struct TcParams {
     int k_splits;   // single-CTA kernel: K ranges per output tile (1: no split)
     float* partials;  // k_splits > 1: fp32 [k_splits][M_cap][N] partial sums
     uint64_t timeout_ns;
+    // transpose_padding_rebuild fused into the epilogue (pair kernel only): output row r
+    // goes to padded row b * scatter_pad_len + r - scatter_cu[b] of a [batch, pad_len, N] tensor
+    const int32_t* scatter_cu;
+    int scatter_batch, scatter_pad_len;
 };
+
+// Destination row of packed row `row` (its padded position when the epilogue scatters).
+__device__ __forceinline__ int64_t out_row_of(const TcParams& p, int row) {
+    if (p.scatter_cu == nullptr) return row;
+    const int b = owner_of(p.scatter_cu, p.scatter_batch, row);
+    return (int64_t)b * p.scatter_pad_len + (row - __ldg(p.scatter_cu + b));
+}
 
 __device__ __forceinline__ void tile_mn(int t, int num_m, int num_n, int group_m, int& m, int& n) {
     const int per_group = group_m * num_n;
@@ -106,8 +117,8 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
 // Bias, optional GELU, optional residual (already loaded by the caller into `res`),
 // one rounding to T, 64-byte store of 32 consecutive columns of one row.
 template <typename T, int EPI>
-__device__ __forceinline__ void epilogue_store32(const uint32_t* acc, const uint4* res, const TcParams& p, int row,
-                                                 int col0) {
+__device__ __forceinline__ void epilogue_store32(const uint32_t* acc, const uint4* res, const TcParams& p,
+                                                 int64_t out_row, int col0) {
     float v[32];
 #pragma unroll
     for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(acc[j]);
@@ -146,7 +157,7 @@ __device__ __forceinline__ void epilogue_store32(const uint32_t* acc, const uint
             }
         }
     }
-    uint4* op = reinterpret_cast<uint4*>(static_cast<T*>(p.out) + (int64_t)row * p.N + col0);
+    uint4* op = reinterpret_cast<uint4*>(static_cast<T*>(p.out) + out_row * p.N + col0);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         uint4 o;
@@ -175,6 +186,7 @@ __device__ __forceinline__ void drain_256(uint32_t tbase, const TcParams& p, int
     uint32_t r[2][32];
     uint4 res[2][4];
     const bool row_ok = row < M;
+    const int64_t out_row = row_ok ? out_row_of(p, row) : 0;
     tmem_ld_x16(tbase, r[0]);
     tmem_ld_x16(tbase + 16, r[0] + 16);
     load_residual32<T, EPI>(p, row, col_base, row_ok && col_base < p.N, res[0]);
@@ -189,7 +201,7 @@ __device__ __forceinline__ void drain_256(uint32_t tbase, const TcParams& p, int
             load_residual32<T, EPI>(p, row, coln, row_ok && coln < p.N, res[cur ^ 1]);
         }
         const int col0 = col_base + c * 32;
-        if (row_ok && col0 < p.N) epilogue_store32<T, EPI>(r[cur], res[cur], p, row, col0);
+        if (row_ok && col0 < p.N) epilogue_store32<T, EPI>(r[cur], res[cur], p, out_row, col0);
     }
 }
 
@@ -212,8 +224,8 @@ __device__ __forceinline__ uint32_t stage_off(int row, int chunk) {
 template <typename T, int EPI>
 __device__ __forceinline__ bool drain_256_staged(uint32_t tbase, const TcParams& p, const CUtensorMap* tmO,
                                                  const CUtensorMap* tmR, uint8_t* sbuf, uint64_t* rbar,
-                                                 uint32_t& rpar, int row_base, int col_base, uint32_t tempty_cluster,
-                                                 const volatile int* abort_flag) {
+                                                 uint32_t& rpar, int row_base, int out_row_base, int col_base,
+                                                 uint32_t tempty_cluster, const volatile int* abort_flag) {
     const int lane = threadIdx.x & 31;
     uint32_t r[2][32];
     bool ok = true;
@@ -316,7 +328,7 @@ __device__ __forceinline__ bool drain_256_staged(uint32_t tbase, const TcParams&
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-            tma_store_2d(tmO, buf, col0, row_base);
+            tma_store_2d(tmO, buf, col0, out_row_base);
             bulk_commit();
         }
     }
@@ -823,8 +835,18 @@ __global__ void __launch_bounds__(PairCfg<MT>::THREADS, 1)
                 const int row_base = (mt * MT + i) * PBM + (int)rank * 128 + q * 32;
                 const uint32_t tbase =
                     tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(slot * C::SLOT_COLS + i * PBN);
-                if (row_base + 32 <= M) {
-                    ok = drain_256_staged<T, EPI>(tbase, p, &tmO, &tmR, sbuf, rb, rpar, row_base, n * PBN,
+                // a 32-row box is one TMA store when its rows are valid and (scattering)
+                // lie in one sequence, so that their padded rows are consecutive too
+                bool box = row_base + 32 <= M;
+                int out_base = row_base;
+                if (box && p.scatter_cu != nullptr) {
+                    const int b = owner_of(p.scatter_cu, p.scatter_batch, row_base);
+                    const int start = __ldg(p.scatter_cu + b);
+                    box = row_base + 32 <= __ldg(p.scatter_cu + b + 1);
+                    out_base = b * p.scatter_pad_len + (row_base - start);
+                }
+                if (box) {
+                    ok = drain_256_staged<T, EPI>(tbase, p, &tmO, &tmR, sbuf, rb, rpar, row_base, out_base, n * PBN,
                                                   tempty_cluster, abort_flag);
                     handed_back = ok;
                 } else {
@@ -895,6 +917,12 @@ static CUresult make_tmap_io(CUtensorMap* m, int dtype, const void* ptr, int64_t
     return fn(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
               CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
+
+// Single-CTA tiles for a GEMM whose rows fit in one 128-row tile (the skinny,
+// weight-streaming case): more CTAs stream weights than with 256-row pair tiles.
+static bool use_single_cta(const GemmArgs& a) { return a.M_cap <= TBM; }
+
+bool gemm_tc_scatter_ok(const GemmArgs& a) { return gemm_tc_supported(a) && !use_single_cta(a); }
 
 bool gemm_tc_supported(const GemmArgs& a) {
     if (a.dtype != ENERGON_F16 && a.dtype != ENERGON_BF16) return false;
@@ -969,9 +997,6 @@ static cudaError_t tc2_dispatch(int epi, const CUtensorMap& ta, const CUtensorMa
     }
 }
 
-// Single-CTA tiles for a GEMM whose rows fit in one 128-row tile (the skinny,
-// weight-streaming case): more CTAs stream weights than with 256-row pair tiles.
-static bool use_single_cta(const GemmArgs& a) { return a.M_cap <= TBM; }
 
 cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st, char* err, size_t errlen) {
     const bool single = use_single_cta(a);
@@ -995,7 +1020,14 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st, char* err, size_t
     p.timeout_ns = a.timeout_ns;
     p.k_splits = 1;
     p.partials = nullptr;
+    p.scatter_cu = a.scatter_cu;
+    p.scatter_batch = a.scatter_batch;
+    p.scatter_pad_len = a.scatter_pad_len;
     const bool bf = a.dtype == ENERGON_BF16;
+    if (single && a.scatter_cu != nullptr) {
+        if (err) snprintf(err, errlen, "scattering epilogue needs the CTA-pair path (more than %d rows)", TBM);
+        return cudaErrorInvalidValue;
+    }
     if (!single) {
         // Pair tiles of two row tiles (512 x 256) once the buffer can hold two: every
         // staged weight panel then feeds 512 rows.
@@ -1009,7 +1041,8 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st, char* err, size_t
         // stores and residual loads.  Only boxes of rows below the live row count are
         // ever copied, so the maps may span the whole buffer capacity.
         CUtensorMap to, tr;
-        CUresult r3 = make_tmap_io(&to, a.dtype, a.out, a.N, a.M_cap);
+        const int64_t out_rows = a.scatter_cu ? (int64_t)a.scatter_batch * a.scatter_pad_len : a.M_cap;
+        CUresult r3 = make_tmap_io(&to, a.dtype, a.out, a.N, out_rows);
         CUresult r4 = a.epilogue == EPI_BIAS_RESIDUAL ? make_tmap_io(&tr, a.dtype, a.residual, a.N, a.M_cap) : r3;
         if (a.epilogue != EPI_BIAS_RESIDUAL) tr = to;
         if (r3 != CUDA_SUCCESS || r4 != CUDA_SUCCESS) {

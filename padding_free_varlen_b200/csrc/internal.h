@@ -29,9 +29,22 @@ cudaError_t launch_transpose_remove(const void* heads, const int32_t* cu, int ba
                                     int n_heads, int64_t head_bytes, int64_t packed_rows_cap, void* packed,
                                     cudaStream_t st);
 
+// Zero the pad rows (s >= cu[b+1] - cu[b]) of padded [batch, pad_len] rows of row_bytes.
+cudaError_t launch_zero_pads(const int32_t* cu, int batch, int pad_len, int64_t row_bytes, void* padded,
+                             cudaStream_t st);
+
+// LayerNorm gather (transpose_padding_remove fused into a LayerNorm): with cu set, row
+// r of the output reads padded row (b, r - cu[b]) of x [batch, pad_len, H] and, with
+// copy set, also writes that raw row to copy[r].
+struct LnGather {
+    const int32_t* cu = nullptr;
+    int batch = 0, pad_len = 0;
+    void* copy = nullptr;
+};
 // LayerNorm over rows [0, min(*d_rows, rows_cap)) of x [rows_cap, H] -> y.
 cudaError_t launch_layernorm(int dtype, const void* x, const void* g, const void* b, void* y, const int32_t* d_rows,
-                             int rows_cap, int H, float eps, const int32_t* status, cudaStream_t st);
+                             int rows_cap, int H, float eps, const int32_t* status, cudaStream_t st,
+                             const LnGather& gth = LnGather());
 
 // Epilogue variants of the GEMM y = A W^T + bias (+ GELU) (+ residual).
 enum Epilogue { EPI_BIAS = 0, EPI_BIAS_GELU = 1, EPI_BIAS_RESIDUAL = 2 };
@@ -52,10 +65,16 @@ struct GemmArgs {
     int gelu_tanh;
     int32_t* status;
     uint64_t timeout_ns;
+    // Optional transpose_padding_rebuild in the epilogue: output row r is stored at padded
+    // row b * scatter_pad_len + r - scatter_cu[b] of out [scatter_batch, scatter_pad_len, N].
+    const int32_t* scatter_cu = nullptr;
+    int scatter_batch = 0, scatter_pad_len = 0;
 };
 
 // True when the tcgen05 path can run this GEMM (16-bit types, alignment, tile multiples).
 bool gemm_tc_supported(const GemmArgs& a);
+// True when it runs on the CTA-pair kernel, the one whose epilogue can scatter.
+bool gemm_tc_scatter_ok(const GemmArgs& a);
 cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st, char* err, size_t errlen);
 cudaError_t launch_gemm_simt(const GemmArgs& a, cudaStream_t st);
 

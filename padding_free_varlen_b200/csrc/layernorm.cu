@@ -7,6 +7,11 @@
 // One thread block per row (grid-stride over the device-side row count).  For
 // 16-bit rows of up to 16384 elements each thread keeps its slice in registers
 // as 16-byte vectors, so the row is read from HBM once and written once.
+//
+// Gather form (transpose_padding_remove fused into the first LayerNorm): packed
+// row r reads padded row (b, r - cu[b]) of a [batch, pad_len, H] tensor and also
+// writes that raw row to `copy` (the packed residual stream), so the padded input
+// is read once for both.
 #include "common.cuh"
 #include "internal.h"
 
@@ -26,16 +31,31 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
     return t;
 }
 
+// Source row of packed row r: itself, or (gather) padded row (b, r - cu[b]); -1 if
+// the offsets put it outside the padded tensor.
+__device__ __forceinline__ int64_t ln_src_row(const LnGather& gth, int r) {
+    if (gth.cu == nullptr) return r;
+    const int b = owner_of(gth.cu, gth.batch, r);
+    const int64_t s = (int64_t)r - __ldg(gth.cu + b);
+    return (s >= 0 && s < gth.pad_len) ? (int64_t)b * gth.pad_len + s : -1;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256) ln_generic_kernel(const T* __restrict__ x, const T* __restrict__ g,
                                                          const T* __restrict__ bb, T* __restrict__ y,
                                                          const int32_t* d_rows, int rows_cap, int H, float eps,
-                                                         const int32_t* status) {
+                                                         const int32_t* status, LnGather gth) {
     __shared__ float red[32];
     if (status_bad(status)) return;
     const int rows = min(*d_rows, rows_cap);
     for (int r = blockIdx.x; r < rows; r += gridDim.x) {
-        const T* xr = x + (int64_t)r * H;
+        const int64_t src = ln_src_row(gth, r);
+        if (src < 0) continue;
+        const T* xr = x + src * H;
+        if (gth.copy != nullptr) {
+            T* cr = static_cast<T*>(gth.copy) + (int64_t)r * H;
+            for (int k = threadIdx.x; k < H; k += blockDim.x) cr[k] = xr[k];
+        }
         float s = 0.0f;
         for (int k = threadIdx.x; k < H; k += blockDim.x) s += to_f(xr[k]);
         const float mean = block_sum(s, red) / H;
@@ -57,13 +77,16 @@ template <typename T, int VPT>
 __global__ void __launch_bounds__(256) ln_vec_kernel(const T* __restrict__ x, const T* __restrict__ g,
                                                      const T* __restrict__ bb, T* __restrict__ y,
                                                      const int32_t* d_rows, int rows_cap, int H, float eps,
-                                                     const int32_t* status) {
+                                                     const int32_t* status, LnGather gth) {
     __shared__ float red[32];
     if (status_bad(status)) return;
     const int rows = min(*d_rows, rows_cap);
     const int nvec = H / 8;
+    uint4* copy = static_cast<uint4*>(gth.copy);
     for (int r = blockIdx.x; r < rows; r += gridDim.x) {
-        const uint4* xr = reinterpret_cast<const uint4*>(x + (int64_t)r * H);
+        const int64_t src = ln_src_row(gth, r);
+        if (src < 0) continue;
+        const uint4* xr = reinterpret_cast<const uint4*>(x + src * H);
         uint4 v[VPT];
         float s = 0.0f;
 #pragma unroll
@@ -71,6 +94,7 @@ __global__ void __launch_bounds__(256) ln_vec_kernel(const T* __restrict__ x, co
             const int idx = i * blockDim.x + threadIdx.x;
             if (idx < nvec) {
                 v[i] = xr[idx];
+                if (copy != nullptr) copy[(int64_t)r * nvec + idx] = v[i];
                 const uint32_t* w = reinterpret_cast<const uint32_t*>(&v[i]);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
@@ -120,22 +144,23 @@ __global__ void __launch_bounds__(256) ln_vec_kernel(const T* __restrict__ x, co
 
 template <typename T>
 static cudaError_t ln_dispatch(const void* x, const void* g, const void* b, void* y, const int32_t* d_rows,
-                               int rows_cap, int H, float eps, const int32_t* status, cudaStream_t st) {
+                               int rows_cap, int H, float eps, const int32_t* status, const LnGather& gth,
+                               cudaStream_t st) {
     const int grid = rows_cap < 8 * device_sm_count() ? (rows_cap > 0 ? rows_cap : 1) : 8 * device_sm_count();
     const T *xp = (const T*)x, *gp = (const T*)g, *bp = (const T*)b;
     T* yp = (T*)y;
-    const uintptr_t al = (uintptr_t)x | (uintptr_t)g | (uintptr_t)b | (uintptr_t)y;
+    const uintptr_t al = (uintptr_t)x | (uintptr_t)g | (uintptr_t)b | (uintptr_t)y | (uintptr_t)gth.copy;
     const int nvec = H / 8;
     const int vpt = (nvec + 255) / 256;
     if (sizeof(T) == 2 && H % 8 == 0 && al % 16 == 0 && vpt >= 1 && vpt <= 8) {
         switch (vpt) {
 #define LN_CASE(V) \
-    case V: ln_vec_kernel<T, V><<<grid, 256, 0, st>>>(xp, gp, bp, yp, d_rows, rows_cap, H, eps, status); break;
+    case V: ln_vec_kernel<T, V><<<grid, 256, 0, st>>>(xp, gp, bp, yp, d_rows, rows_cap, H, eps, status, gth); break;
             LN_CASE(1) LN_CASE(2) LN_CASE(3) LN_CASE(4) LN_CASE(5) LN_CASE(6) LN_CASE(7) LN_CASE(8)
 #undef LN_CASE
         }
     } else {
-        ln_generic_kernel<T><<<grid, 256, 0, st>>>(xp, gp, bp, yp, d_rows, rows_cap, H, eps, status);
+        ln_generic_kernel<T><<<grid, 256, 0, st>>>(xp, gp, bp, yp, d_rows, rows_cap, H, eps, status, gth);
     }
     return cudaGetLastError();
 }
@@ -143,19 +168,21 @@ static cudaError_t ln_dispatch(const void* x, const void* g, const void* b, void
 // The vector kernel only exists for 16-bit types; fp32 always takes the generic one.
 template <>
 cudaError_t ln_dispatch<float>(const void* x, const void* g, const void* b, void* y, const int32_t* d_rows,
-                               int rows_cap, int H, float eps, const int32_t* status, cudaStream_t st) {
+                               int rows_cap, int H, float eps, const int32_t* status, const LnGather& gth,
+                               cudaStream_t st) {
     const int grid = rows_cap < 8 * device_sm_count() ? (rows_cap > 0 ? rows_cap : 1) : 8 * device_sm_count();
     ln_generic_kernel<float><<<grid, 256, 0, st>>>((const float*)x, (const float*)g, (const float*)b, (float*)y,
-                                                   d_rows, rows_cap, H, eps, status);
+                                                   d_rows, rows_cap, H, eps, status, gth);
     return cudaGetLastError();
 }
 
 cudaError_t launch_layernorm(int dtype, const void* x, const void* g, const void* b, void* y, const int32_t* d_rows,
-                             int rows_cap, int H, float eps, const int32_t* status, cudaStream_t st) {
+                             int rows_cap, int H, float eps, const int32_t* status, cudaStream_t st,
+                             const LnGather& gth) {
     switch (dtype) {
-    case ENERGON_F32: return ln_dispatch<float>(x, g, b, y, d_rows, rows_cap, H, eps, status, st);
-    case ENERGON_F16: return ln_dispatch<__half>(x, g, b, y, d_rows, rows_cap, H, eps, status, st);
-    case ENERGON_BF16: return ln_dispatch<__nv_bfloat16>(x, g, b, y, d_rows, rows_cap, H, eps, status, st);
+    case ENERGON_F32: return ln_dispatch<float>(x, g, b, y, d_rows, rows_cap, H, eps, status, gth, st);
+    case ENERGON_F16: return ln_dispatch<__half>(x, g, b, y, d_rows, rows_cap, H, eps, status, gth, st);
+    case ENERGON_BF16: return ln_dispatch<__nv_bfloat16>(x, g, b, y, d_rows, rows_cap, H, eps, status, gth, st);
     }
     return cudaErrorInvalidValue;
 }

@@ -95,17 +95,6 @@ cudaError_t launch_padded_starts(int batch, int pad_len, int32_t* cu_pad, const 
 
 // ------------------------------------------------------------------ remove / rebuild
 
-// Largest b in [0, batch) with cu[b] <= r (the sequence that owns packed row r).
-__device__ __forceinline__ int owner_of(const int32_t* __restrict__ cu, int batch, int64_t r) {
-    int lo = 0, hi = batch - 1;
-    while (lo < hi) {
-        int mid = (lo + hi + 1) >> 1;
-        if (__ldg(cu + mid) <= r) lo = mid;
-        else hi = mid - 1;
-    }
-    return lo;
-}
-
 template <typename V, int UNROLL>
 __device__ __forceinline__ void warp_copy_row(const V* __restrict__ src, V* __restrict__ dst, int64_t nvec, int lane) {
     for (int64_t base = lane; base < nvec; base += 32 * UNROLL) {
@@ -212,6 +201,33 @@ cudaError_t launch_rebuild(const void* packed, const int32_t* starts, const int3
         rebuild_kernel<uint8_t, 8><<<grid, 256, 0, st>>>((const uint8_t*)packed, starts, lens_cu, batch, pad_len,
                                                          row_bytes, packed_rows_cap, (uint8_t*)padded);
     }
+    return cudaGetLastError();
+}
+
+// Zero the pad rows (s >= len_b) of a padded [batch, pad_len] tensor; valid rows untouched.
+template <typename V>
+__global__ void __launch_bounds__(256) zero_pads_kernel(const int32_t* __restrict__ cu, int batch, int pad_len,
+                                                        int64_t row_vecs, V* __restrict__ padded) {
+    const int lane = threadIdx.x & 31;
+    const int64_t rows = (int64_t)batch * pad_len;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
+        const int b = (int)(r / pad_len);
+        const int s = (int)(r - (int64_t)b * pad_len);
+        if (s >= __ldg(cu + b + 1) - __ldg(cu + b)) warp_zero_row<V>(padded + r * row_vecs, row_vecs, lane);
+    }
+}
+
+cudaError_t launch_zero_pads(const int32_t* cu, int batch, int pad_len, int64_t row_bytes, void* padded,
+                             cudaStream_t st) {
+    if (batch <= 0 || pad_len <= 0 || row_bytes == 0) return cudaSuccess;
+    const int grid = row_grid((int64_t)batch * pad_len);
+    if (row_bytes % 16 == 0 && reinterpret_cast<uintptr_t>(padded) % 16 == 0)
+        zero_pads_kernel<uint4><<<grid, 256, 0, st>>>(cu, batch, pad_len, row_bytes / 16, (uint4*)padded);
+    else if (row_bytes % 4 == 0 && reinterpret_cast<uintptr_t>(padded) % 4 == 0)
+        zero_pads_kernel<uint32_t><<<grid, 256, 0, st>>>(cu, batch, pad_len, row_bytes / 4, (uint32_t*)padded);
+    else
+        zero_pads_kernel<uint8_t><<<grid, 256, 0, st>>>(cu, batch, pad_len, row_bytes, (uint8_t*)padded);
     return cudaGetLastError();
 }
 

@@ -250,24 +250,35 @@ def test_stack_invalid_lengths_and_empty_batch():
         assert st == 0 and (out.view(torch.int16) == 0).all()
 
 
-def test_stack_modes_launch_their_own_schedules():
+@pytest.mark.parametrize("S", [16, 64])
+def test_stack_modes_launch_their_own_schedules(S):
     """The three modes agree on valid rows by design, so their schedules are told apart by
-    the launch trace: packing once around the stack (1), never (0), or around every MLP (2)."""
+    the launch trace.  Mode 1 packs inside the first LayerNorm and, when the last FFN2 runs
+    on the CTA-pair GEMM (more than 128 buffer rows), scatters back inside its epilogue;
+    mode 0 never packs; mode 2 packs around every MLP with the standalone operators."""
     shape = synth.LayerShape(256, 2, 512)
-    lengths = np.array([5, 16, 9], np.int32)
-    x = synth.normal((3, 16, 256), 3, synth.TID_X, synth.F16)
+    lengths = np.array([5, S, 9], np.int32)
+    x = synth.normal((3, S, 256), 3, synth.TID_X, synth.F16)
     L = 3
-    want = {1: {"remove_padding": 1, "rebuild_padding": 1, "padded_starts": 0},
-            0: {"remove_padding": 0, "rebuild_padding": 1, "padded_starts": 1},
-            2: {"remove_padding": L, "rebuild_padding": L, "padded_starts": 1}}
+    pair = 3 * S > 128
+    want = {1: {"remove_padding": 0, "layernorm_remove": 1, "zero_pads": 1, "padded_starts": 0,
+                "rebuild_padding": 0 if pair else 1, "gemm_ffn2_rebuild": 1 if pair else 0},
+            0: {"remove_padding": 0, "layernorm_remove": 0, "rebuild_padding": 1, "padded_starts": 1,
+                "gemm_ffn2_rebuild": 0},
+            2: {"remove_padding": L, "layernorm_remove": 0, "rebuild_padding": L, "padded_starts": 1,
+                "gemm_ffn2_rebuild": 0}}
+    outs = {}
     for mode, counts in want.items():
         capi.energon_trace_start()
-        _, st, _ = stack_run(synth.F16, shape, L, x, lengths, 3, NONZERO, mode)
+        outs[mode], st, _ = stack_run(synth.F16, shape, L, x, lengths, 3, NONZERO, mode)
         trace = capi.energon_trace_stop()
         assert st == 0
         got = {k: trace.get(k, (0, 0.0))[0] for k in counts}
         assert got == counts, (mode, trace)
-        assert trace["gemm_qkv"][0] == trace["gemm_ffn2"][0] == L
+        n_ffn2 = trace.get("gemm_ffn2", (0, 0.0))[0] + trace.get("gemm_ffn2_rebuild", (0, 0.0))[0]
+        assert trace["gemm_qkv"][0] == n_ffn2 == L
+    assert torch.equal(outs[1].view(torch.int16), outs[0].view(torch.int16))
+    assert torch.equal(outs[1].view(torch.int16), outs[2].view(torch.int16))
 
 
 @pytest.mark.parametrize("mode", [0, 1, 2])
