@@ -270,6 +270,53 @@ ENERGON_API int energon_rce_remove_padding_noalloc(const void* padded, const int
                                                    int pad_len, int hidden, int elem_bytes, void* packed,
                                                    int32_t* d_status, void* stream);
 
+/*
+ * Dynamic batching of a request queue (host runtime; no device memory, no GPU
+ * needed).  The QbitAI article's "Serving" section and the EnergonAI README's
+ * "Batching" section: queued requests are packed into batches as the machine's
+ * performance suits best, and the batch of highest priority - from the waiting
+ * time, the batch size and the batch's length after padding - runs first,
+ * avoiding starvation; the method follows TurboTransformer's dynamic-programming
+ * batch scheduler and is compared against FIFO packing.  The pages give no
+ * formula; the reading implemented here:
+ *   packing   requests sorted by (length, arrival, index) are cut into
+ *             consecutive groups of at most max_batch minimising the summed cost
+ *             cost(b, s) = cost_table[(b - 1) * table_max_len + (s - 1)] of b
+ *             sequences padded to s tokens (measured on the machine; any positive
+ *             unit); the scan over group starts keeps the first minimum;
+ *   priority  (tokens of the group) / cost(size, longest length)
+ *             * (1 + (now_s - earliest arrival in the group) / age_scale_s).
+ *   reqs       [n] requests (length in [1, table_max_len], finite arrival_s)
+ *   cost_table [max_batch * table_max_len] doubles, finite and > 0 (only rows
+ *              b <= min(max_batch, n) are read)
+ *   group_of   out [n]: group of each request; groups are numbered in ascending
+ *              length order
+ *   n_groups   out: number of groups
+ *   order      out [n] (first *n_groups used): group indices by descending
+ *              priority, ties by ascending index
+ * All buffers are host memory owned by the caller.  Errors (before any output
+ * is written): NULL pointer, n < 0, max_batch or table_max_len < 1, a length out
+ * of range, a non-finite time, age_scale_s <= 0, a bad cost entry ->
+ * ENERGON_ERR_INVALID_ARGUMENT.
+ */
+typedef struct {
+    int32_t length;   /* valid tokens of the request */
+    double arrival_s; /* arrival time, seconds on any common clock */
+} energon_request;
+
+ENERGON_API int energon_sched_plan(const energon_request* reqs, int n, double now_s, int max_batch,
+                       const double* cost_table, int table_max_len, double age_scale_s,
+                       int32_t* group_of, int32_t* n_groups, int32_t* order);
+
+/*
+ * FIFO packing, the pages' comparison: requests in arrival order (ties by
+ * index) cut into consecutive groups of max_batch.  group_of [n] and n_groups
+ * out (host memory).  Errors: NULL pointer, n < 0, max_batch < 1, a non-finite
+ * time -> ENERGON_ERR_INVALID_ARGUMENT.
+ */
+ENERGON_API int energon_sched_fifo(const energon_request* reqs, int n, int max_batch, int32_t* group_of,
+                       int32_t* n_groups);
+
 /* Message describing the last failed call on this thread ("" if none). */
 ENERGON_API const char* energon_last_error(void);
 

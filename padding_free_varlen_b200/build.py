@@ -19,7 +19,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD_DIR = os.path.join(HERE, "_build")
 LIB_PATH = os.path.join(HERE, "libenergon_rce.so")
-SOURCES = ["rce.cu", "layernorm.cu", "gemm_simt.cu", "gemm_tc.cu", "attention.cu", "attention_tc.cu", "noalloc.cu", "capi.cu"]
+SOURCES = ["rce.cu", "layernorm.cu", "gemm_simt.cu", "gemm_tc.cu", "attention.cu", "attention_tc.cu", "noalloc.cu", "scheduler.cu", "capi.cu"]
 HEADERS = ["common.cuh", "internal.h"]
 PUBLIC_HEADERS = [os.path.join(ROOT, "include", "energon_rce.h")]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -36,7 +36,8 @@ EXPORTED = ("energon_rce_offsets", "energon_rce_remove_padding", "energon_rce_re
             "energon_workspace_bytes", "energon_layer_forward", "energon_stack_forward",
             "energon_selftest_bounded_wait", "energon_set_wait_timeout_us", "energon_last_error",
             "energon_trace_start", "energon_trace_stop", "energon_rce_remove_padding_noalloc",
-            "energon_rce_transpose_padding_rebuild", "energon_rce_transpose_padding_remove")
+            "energon_rce_transpose_padding_rebuild", "energon_rce_transpose_padding_remove",
+            "energon_sched_plan", "energon_sched_fifo")
 ENERGON_NOALLOC_MAX_BATCH = 16384
 WEIGHT_FIELDS = ("ln1_g", "ln1_b", "w_qkv", "b_qkv", "w_o", "b_o",
                  "ln2_g", "ln2_b", "w_1", "b_1", "w_2", "b_2")
@@ -55,6 +56,10 @@ class energon_layer_config(ctypes.Structure):
 
 class energon_layer_weights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in WEIGHT_FIELDS]
+
+
+class energon_request(ctypes.Structure):
+    _fields_ = [("length", ctypes.c_int32), ("arrival_s", ctypes.c_double)]
 
 
 class energon_trace_entry(ctypes.Structure):
@@ -88,6 +93,11 @@ def load() -> ctypes.CDLL:
             "energon_trace_start": ([], ci),
             "energon_rce_remove_padding_noalloc": ([vp, vp, ci, ci, ci, ci, vp, vp, vp], ci),
             "energon_trace_stop": ([ctypes.POINTER(energon_trace_entry), ci, ctypes.POINTER(ci)], ci),
+            "energon_sched_plan": ([ctypes.POINTER(energon_request), ci, ctypes.c_double, ci,
+                                    ctypes.POINTER(ctypes.c_double), ci, ctypes.c_double, ctypes.POINTER(ctypes.c_int32),
+                                    ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)], ci),
+            "energon_sched_fifo": ([ctypes.POINTER(energon_request), ci, ci, ctypes.POINTER(ctypes.c_int32),
+                                    ctypes.POINTER(ctypes.c_int32)], ci),
         }
         for name, (args, res) in sigs.items():
             f = getattr(L, name)
@@ -216,6 +226,43 @@ def energon_trace_stop() -> dict:
     n = ctypes.c_int(0)
     _check(load().energon_trace_stop(arr, cap, ctypes.byref(n)), "energon_trace_stop")
     return {arr[i].name.decode(): (arr[i].launches, arr[i].total_ms) for i in range(min(n.value, cap))}
+
+
+def _requests(lengths, arrivals):
+    n = len(lengths)
+    if len(arrivals) != n:
+        raise ValueError("lengths and arrivals differ in size")
+    arr = (energon_request * max(1, n))()
+    for i in range(n):
+        arr[i].length = int(lengths[i])
+        arr[i].arrival_s = float(arrivals[i])
+    return arr, n
+
+
+def energon_sched_plan(lengths, arrivals, now_s, max_batch, cost_table, age_scale_s):
+    """Dynamic batching decision for a queue snapshot (host only).  cost_table: nested
+    [max_batch][table_max_len] of positive costs.  Returns (group_of, order) as lists."""
+    reqs, n = _requests(lengths, arrivals)
+    rows = len(cost_table)
+    width = len(cost_table[0]) if rows else 0
+    flat = (ctypes.c_double * max(1, rows * width))(*[float(v) for row in cost_table for v in row])
+    group_of = (ctypes.c_int32 * max(1, n))()
+    order = (ctypes.c_int32 * max(1, n))()
+    ng = ctypes.c_int32(0)
+    if rows < min(max_batch, n):
+        raise ValueError("cost_table has fewer rows than the batch sizes it must price")
+    _check(load().energon_sched_plan(reqs, n, float(now_s), int(max_batch), flat, width, float(age_scale_s),
+                                     group_of, ctypes.byref(ng), order), "energon_sched_plan")
+    return [group_of[i] for i in range(n)], [order[g] for g in range(ng.value)]
+
+
+def energon_sched_fifo(arrivals, max_batch):
+    """FIFO packing: group_of for requests in arrival order (host only)."""
+    reqs, n = _requests([1] * len(arrivals), arrivals)
+    group_of = (ctypes.c_int32 * max(1, n))()
+    ng = ctypes.c_int32(0)
+    _check(load().energon_sched_fifo(reqs, n, int(max_batch), group_of, ctypes.byref(ng)), "energon_sched_fifo")
+    return [group_of[i] for i in range(n)]
 
 
 # ----------------------------------------------------------------------------- struct helpers
