@@ -50,6 +50,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-padded", action="store_true")
     ap.add_argument("--no-transpose", action="store_true")
+    ap.add_argument("--no-batching", action="store_true")
     ap.add_argument("--layers", type=int, default=0, help="override the workload's layer count (profiling)")
     return ap.parse_args()
 
@@ -454,6 +455,12 @@ def run_energon(args, dist: Dist):
                          "ms_per_launch": ms_t, "standalone": True}
         del pk
 
+    # ---- dynamic batching of a request stream (the pages' comparison against FIFO packing,
+    # every batch padded to its longest request) on this machine's measured costs
+    batching = None
+    if not args.no_batching and args.workload == "gpt3_stack_half_pad" and dist.world == 1:
+        batching = run_batching(args, capi, synth, cfg, tables, L, H, tdt, dev, stream, timed, d_in, st)
+
     launches = sum(v[0] for v in trace.values())
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": dist.world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
@@ -461,11 +468,77 @@ def run_energon(args, dist: Dist):
             "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights)",
             "config": config_of(wl, S, T, dist.world), "roofline": roofline, "roofline_memory_kernels": aux,
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clk,
-            "padded_path": padded, "transpose_forms": transpose, "kernels": per_kernel, "setup_s": setup_s}
+            "padded_path": padded, "transpose_forms": transpose, "dynamic_batching": batching,
+            "kernels": per_kernel, "setup_s": setup_s}
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
     del tables
     dist.done()
+
+
+def run_batching(args, capi, synth, cfg, tables, L, H, tdt, dev, stream, timed, pool, st):
+    """Serves 256 requests (lengths U[1, 256], all queued at once) in batches of at most 64:
+    FIFO packing vs the dynamic-programming scheduler (energon_sched_plan), each batch padded
+    to its longest request and run (a) on every padded row, as in the pages' comparison, and
+    (b) with the padding eliminated.  The scheduler's cost table is this machine's: the
+    padded stack timed at two shapes, fitted as c0 + c1 * batch * padded length.  Request
+    activations are rows of the bench batch (the values do not change the work)."""
+    import torch
+    n_req, max_b, max_s = 256, 64, 256
+    lengths = [int(v) for v in synth.uniform_int(n_req, 1, max_s, 20260006, synth.TID_LENGTHS)]
+    arrivals = [0.0] * n_req
+    ws_bytes = capi.energon_workspace_bytes(cfg, max_b, max_s)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    nb = pool.shape[0]
+
+    def make_batch(members):
+        s_pad = max(lengths[i] for i in members)
+        x = torch.stack([pool[i % nb, :s_pad] for i in members]).contiguous()
+        lens = torch.tensor([lengths[i] for i in members], dtype=torch.int32, device=dev)
+        return x, lens, torch.empty_like(x), s_pad
+
+    def run(batches, mode):
+        def go():
+            for x, lens, out, s_pad in batches:
+                capi.energon_stack_forward(cfg, tables, L, x, lens, x.shape[0], s_pad, mode, out, st, ws, ws_bytes,
+                                           stream)
+        return timed(go, 1)
+
+    # machine costs of the padded stack
+    pts = []
+    for b, s_len in ((max_b, max_s), (8, 32)):
+        x = torch.stack([pool[i % nb, :s_len] for i in range(b)]).contiguous()
+        lens = torch.full((b,), s_len, dtype=torch.int32, device=dev)
+        out = torch.empty_like(x)
+        f = lambda: capi.energon_stack_forward(cfg, tables, L, x, lens, b, s_len, 0, out, st, ws, ws_bytes, stream)
+        f()
+        pts.append((b * s_len, timed(f, 1) / 1e3))
+    c1 = max((pts[0][1] - pts[1][1]) / (pts[0][0] - pts[1][0]), 1e-12)
+    c0 = max(pts[0][1] - c1 * pts[0][0], 1e-6)
+    table = [[c0 + c1 * b * s_len for s_len in range(1, max_s + 1)] for b in range(1, max_b + 1)]
+
+    fifo_of = capi.energon_sched_fifo(arrivals, max_b)
+    fifo_groups = [[i for i in range(n_req) if fifo_of[i] == g] for g in range(max(fifo_of) + 1)]
+    plan_of, order = capi.energon_sched_plan(lengths, arrivals, 0.0, max_b, table, 1.0)
+    dyn_groups = [[i for i in range(n_req) if plan_of[i] == g] for g in order]
+    tokens = sum(lengths)
+    res = {"requests": n_req, "max_batch": max_b, "valid_tokens": tokens,
+           "lengths": "U[1, 256], seed 20260006, all queued at time 0",
+           "cost_model": {"c0_s": c0, "c1_s_per_padded_token": c1, "fitted_on": "padded stack at 64 x 256 and 8 x 32"}}
+    for name, groups in (("fifo", fifo_groups), ("dynamic", dyn_groups)):
+        batches = [make_batch(g) for g in groups]
+        padded_tokens = sum(b[0].shape[0] * b[3] for b in batches)
+        for mode, tag in ((0, "padded"), (1, "packed")):
+            ms = run(batches, mode)
+            res[f"{name}_{tag}"] = {"tokens_per_s": tokens / (ms / 1e3), "ms": ms, "batches": len(batches),
+                                    "padded_tokens": padded_tokens}
+        del batches
+    res["gain_dynamic_over_fifo_padded"] = res["dynamic_padded"]["tokens_per_s"] / res["fifo_padded"]["tokens_per_s"]
+    res["gain_packed_fifo_over_fifo_padded"] = res["fifo_packed"]["tokens_per_s"] / res["fifo_padded"]["tokens_per_s"]
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {int(st.item())} after the batching runs")
+    del ws
+    return res
 
 
 def main():

@@ -61,14 +61,17 @@ __device__ __forceinline__ float gelu_f(float v, bool tanh_form) {
     return 0.5f * v * (1.0f + erff(v * 0.7071067811865476f));
 }
 
-// GELU tanh form for results that are rounded to a 16-bit type: tanh(u) taken as
-// 1 - 2 / (exp(2u) + 1) with the fast exponential and division intrinsics.  Its
-// error (about 1e-5 relative, 1e-7 absolute near 0) is far below the 2^-11
-// rounding of the 16-bit output; fp32 outputs use gelu_f.
+// tanh-form GELU for 16-bit outputs.  0.5 v (1 + tanh(u)) equals v / (1 + exp(-2u))
+// exactly, u = sqrt(2/pi) (v + 0.044715 v^3); the quotient form needs one fast
+// exponential and one fast division and never subtracts nearly equal numbers (for
+// v << 0 the result is a small quotient, not 1 + t with t near -1).  Its error
+// (a few 1e-6 relative) is far below the 2^-11 rounding of the 16-bit output;
+// fp32 outputs use gelu_f.
 __device__ __forceinline__ float gelu_tanh_fast(float v) {
-    const float u = 0.7978845608028654f * (v + 0.044715f * v * v * v);
-    const float t = 1.0f - __fdividef(2.0f, __expf(2.0f * u) + 1.0f);
-    return 0.5f * v * (1.0f + t);
+    constexpr float k0 = -2.0f * 0.7978845608028654f;              // -2 sqrt(2/pi)
+    constexpr float k1 = -2.0f * 0.7978845608028654f * 0.044715f;
+    const float neg2u = v * fmaf(v * v, k1, k0);
+    return __fdividef(v, 1.0f + __expf(neg2u));
 }
 
 // ----------------------------------------------------------------- status word
