@@ -142,11 +142,26 @@ __global__ void __launch_bounds__(256) ln_vec_kernel(const T* __restrict__ x, co
     }
 }
 
+// Blocks of `kernel` (256 threads) that fit on the GPU at once: the row loop then runs
+// in a single wave of blocks instead of leaving a second wave to start late.
+template <typename K>
+static int resident_blocks(K kernel) {
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, 256, 0) != cudaSuccess || per_sm < 1) {
+        (void)cudaGetLastError();
+        per_sm = 1;
+    }
+    return per_sm * device_sm_count();
+}
+
+static int ln_grid(int rows_cap, int resident) {
+    return rows_cap < resident ? (rows_cap > 0 ? rows_cap : 1) : resident;
+}
+
 template <typename T>
 static cudaError_t ln_dispatch(const void* x, const void* g, const void* b, void* y, const int32_t* d_rows,
                                int rows_cap, int H, float eps, const int32_t* status, const LnGather& gth,
                                cudaStream_t st) {
-    const int grid = rows_cap < 8 * device_sm_count() ? (rows_cap > 0 ? rows_cap : 1) : 8 * device_sm_count();
     const T *xp = (const T*)x, *gp = (const T*)g, *bp = (const T*)b;
     T* yp = (T*)y;
     const uintptr_t al = (uintptr_t)x | (uintptr_t)g | (uintptr_t)b | (uintptr_t)y | (uintptr_t)gth.copy;
@@ -154,13 +169,20 @@ static cudaError_t ln_dispatch(const void* x, const void* g, const void* b, void
     const int vpt = (nvec + 255) / 256;
     if (sizeof(T) == 2 && H % 8 == 0 && al % 16 == 0 && vpt >= 1 && vpt <= 8) {
         switch (vpt) {
-#define LN_CASE(V) \
-    case V: ln_vec_kernel<T, V><<<grid, 256, 0, st>>>(xp, gp, bp, yp, d_rows, rows_cap, H, eps, status, gth); break;
+#define LN_CASE(V)                                                                                      \
+    case V: {                                                                                           \
+        static const int resident = resident_blocks(ln_vec_kernel<T, V>);                               \
+        ln_vec_kernel<T, V><<<ln_grid(rows_cap, resident), 256, 0, st>>>(xp, gp, bp, yp, d_rows, rows_cap, H, \
+                                                                         eps, status, gth);             \
+        break;                                                                                          \
+    }
             LN_CASE(1) LN_CASE(2) LN_CASE(3) LN_CASE(4) LN_CASE(5) LN_CASE(6) LN_CASE(7) LN_CASE(8)
 #undef LN_CASE
         }
     } else {
-        ln_generic_kernel<T><<<grid, 256, 0, st>>>(xp, gp, bp, yp, d_rows, rows_cap, H, eps, status, gth);
+        static const int resident = resident_blocks(ln_generic_kernel<T>);
+        ln_generic_kernel<T><<<ln_grid(rows_cap, resident), 256, 0, st>>>(xp, gp, bp, yp, d_rows, rows_cap, H, eps,
+                                                                         status, gth);
     }
     return cudaGetLastError();
 }
@@ -170,9 +192,9 @@ template <>
 cudaError_t ln_dispatch<float>(const void* x, const void* g, const void* b, void* y, const int32_t* d_rows,
                                int rows_cap, int H, float eps, const int32_t* status, const LnGather& gth,
                                cudaStream_t st) {
-    const int grid = rows_cap < 8 * device_sm_count() ? (rows_cap > 0 ? rows_cap : 1) : 8 * device_sm_count();
-    ln_generic_kernel<float><<<grid, 256, 0, st>>>((const float*)x, (const float*)g, (const float*)b, (float*)y,
-                                                   d_rows, rows_cap, H, eps, status, gth);
+    static const int resident = resident_blocks(ln_generic_kernel<float>);
+    ln_generic_kernel<float><<<ln_grid(rows_cap, resident), 256, 0, st>>>(
+        (const float*)x, (const float*)g, (const float*)b, (float*)y, d_rows, rows_cap, H, eps, status, gth);
     return cudaGetLastError();
 }
 

@@ -205,23 +205,30 @@ cudaError_t launch_rebuild(const void* packed, const int32_t* starts, const int3
 }
 
 // Zero the pad rows (s >= len_b) of a padded [batch, pad_len] tensor; valid rows untouched.
+// The pad rows of one sequence are one contiguous byte range, so blocks (blockIdx.y: the
+// sequence, grid-strided) sweep that range with consecutive 16-byte stores.
 template <typename V>
 __global__ void __launch_bounds__(256) zero_pads_kernel(const int32_t* __restrict__ cu, int batch, int pad_len,
                                                         int64_t row_vecs, V* __restrict__ padded) {
-    const int lane = threadIdx.x & 31;
-    const int64_t rows = (int64_t)batch * pad_len;
-    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
-        const int b = (int)(r / pad_len);
-        const int s = (int)(r - (int64_t)b * pad_len);
-        if (s >= __ldg(cu + b + 1) - __ldg(cu + b)) warp_zero_row<V>(padded + r * row_vecs, row_vecs, lane);
+    V z;
+    memset(&z, 0, sizeof(V));
+    for (int b = blockIdx.y; b < batch; b += gridDim.y) {
+        int len = __ldg(cu + b + 1) - __ldg(cu + b);
+        len = len < 0 ? 0 : (len > pad_len ? pad_len : len);
+        V* dst = padded + ((int64_t)b * pad_len + len) * row_vecs;
+        const int64_t n = (int64_t)(pad_len - len) * row_vecs;
+        for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+            __stcs(dst + i, z);
     }
 }
 
 cudaError_t launch_zero_pads(const int32_t* cu, int batch, int pad_len, int64_t row_bytes, void* padded,
                              cudaStream_t st) {
     if (batch <= 0 || pad_len <= 0 || row_bytes == 0) return cudaSuccess;
-    const int grid = row_grid((int64_t)batch * pad_len);
+    const int gy = batch < 65535 ? batch : 65535;
+    int gx = (4 * device_sm_count() + gy - 1) / gy;  // about four blocks per SM in all
+    if (gx < 1) gx = 1;
+    const dim3 grid(gx, gy);
     if (row_bytes % 16 == 0 && reinterpret_cast<uintptr_t>(padded) % 16 == 0)
         zero_pads_kernel<uint4><<<grid, 256, 0, st>>>(cu, batch, pad_len, row_bytes / 16, (uint4*)padded);
     else if (row_bytes % 4 == 0 && reinterpret_cast<uintptr_t>(padded) % 4 == 0)
