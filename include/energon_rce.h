@@ -49,7 +49,7 @@ extern "C" {
 typedef enum {
     ENERGON_OK = 0,
     ENERGON_ERR_INVALID_ARGUMENT = 1, /* null pointer, negative size, bad enum */
-    ENERGON_ERR_UNSUPPORTED = 2,      /* dtype / shape this build does not run */
+    ENERGON_ERR_UNSUPPORTED = 2,      /* dtype / shape the library does not run */
     ENERGON_ERR_MISALIGNED = 3,       /* a pointer breaks an alignment the path needs */
     ENERGON_ERR_CUDA = 4,             /* a CUDA runtime / launch error */
     ENERGON_ERR_WORKSPACE_TOO_SMALL = 5,

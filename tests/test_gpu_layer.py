@@ -3,7 +3,7 @@
 Two kinds of checks, all through the C ABI:
   * step parity: every step's GPU output (read from the documented workspace
     regions) against the oracle applied to the GPU's own inputs of that step,
-    so each step is judged alone: within one unit in the last place of the
+    so each step is checked alone: within one unit in the last place of the
     storage type plus an fp32-accumulation allowance;
   * end to end: the layer / stack output against the oracle on the original
     inputs, relative Frobenius error <= 5e-3 and max-abs error <= 2e-2 (the
