@@ -229,6 +229,32 @@ def traffic_from_profile() -> int | None:
     return d.get("dram_bytes_per_launch_scaled")
 
 
+def gemm_roofline(H: int, T: int, elem_bytes: int, launches: int, ms_total: float, peaks: dict,
+                  traffic) -> dict:
+    """Roofline object of the four GEMMs of a layer (QKV 3H x H, out-proj H x H, FFN1 4H x H,
+    FFN2 H x 4H) on T rows, averaged per launch.  A launch of T rows does 2 T flop per weight
+    element (T flop per 16-bit weight byte): below the machine's ridge (measured peak flop /
+    measured HBM bytes) it is bound by streaming the weights, and is reported in bytes per
+    second against the HBM rate."""
+    flops_per_launch = 24 * H * H * T / 4
+    weight_bytes_per_launch = 12 * H * H * elem_bytes / 4
+    ms_per_launch = ms_total / max(1, launches)
+    ridge = peaks["tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if flops_per_launch / weight_bytes_per_launch < ridge:
+        achieved = weight_bytes_per_launch * launches / (ms_total / 1e3) / 1e9 if ms_total > 0 else None
+        return {"bound": "hbm", "kernel": "gemm_tc (tcgen05, 4 shapes per layer), weight streaming",
+                "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"] if achieved else None,
+                "peak_note": f"{peaks['source']} HBM copy rate", "traffic": None,
+                "algorithmic_bytes_per_launch": weight_bytes_per_launch, "ms_per_launch": ms_per_launch}
+    achieved = flops_per_launch * launches / (ms_total / 1e3) / 1e12 if ms_total > 0 else None
+    return {"bound": "tensor", "kernel": "gemm_tc (tcgen05, 4 shapes per layer)",
+            "achieved": achieved, "peak": peaks["tflops_sustained"], "unit": "TFLOP/s",
+            "frac": achieved / peaks["tflops_sustained"] if achieved else None,
+            "peak_note": f"{peaks['source']} bf16 sustained (fp16 assumed at the bf16 rate); burst {peaks['tflops']}",
+            "traffic": traffic, "algorithmic_flops_per_launch": flops_per_launch, "ms_per_launch": ms_per_launch}
+
+
 def run_energon(args, dist: Dist):
     import torch
     from padding_free_varlen_b200 import build as cuda_build
@@ -347,33 +373,9 @@ def run_energon(args, dist: Dist):
     gemm_names = ("gemm_qkv", "gemm_out_proj", "gemm_ffn1", "gemm_ffn2", "gemm_ffn2_rebuild")
     g_launch = sum(trace.get(n, (0, 0.0))[0] for n in gemm_names)
     g_ms = sum(trace.get(n, (0, 0.0))[1] for n in gemm_names)
-    flops_per_token_layer = 24 * H * H            # 2*(3H*H + H*H + 4H*H + 4H*H)
-    gemm_flops_per_launch = flops_per_token_layer * T / 4
-    e_w = 2 if tdt != torch.float32 else 4
-    weight_bytes_per_launch = 12 * H * H * e_w / 4   # each layer's weights are read once
     per_kernel = {k: {"launches": v[0], "ms_per_step": v[1] / args.steps,
                       "share": v[1] / max(1e-9, sum(x[1] for x in trace.values()))} for k, v in trace.items()}
-    traffic = traffic_from_profile()
-    # A GEMM of T rows does 2*T flop per weight byte (16-bit): below the machine's ridge
-    # (measured peak flop / measured HBM bytes) it is bound by streaming the weights.
-    ridge = peaks["tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
-    if gemm_flops_per_launch / weight_bytes_per_launch < ridge:
-        achieved = (weight_bytes_per_launch * g_launch) / (g_ms / 1e3) / 1e9 if g_ms > 0 else None
-        roofline = {"bound": "hbm", "kernel": "gemm_tc (tcgen05, 4 shapes per layer), weight streaming",
-                    "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": achieved / peaks["hbm_gbs"] if achieved else None,
-                    "peak_note": f"{peaks['source']} HBM copy rate",
-                    "traffic": None, "algorithmic_bytes_per_launch": weight_bytes_per_launch,
-                    "ms_per_launch": g_ms / max(1, g_launch)}
-    else:
-        achieved = (gemm_flops_per_launch * g_launch) / (g_ms / 1e3) / 1e12 if g_ms > 0 else None
-        roofline = {"bound": "tensor", "kernel": "gemm_tc (tcgen05, 4 shapes per layer)",
-                    "achieved": achieved, "peak": peaks["tflops_sustained"], "unit": "TFLOP/s",
-                    "frac": achieved / peaks["tflops_sustained"] if achieved else None,
-                    "peak_note": f"{peaks['source']} bf16 sustained (fp16 assumed at the bf16 rate); "
-                                 f"burst {peaks['tflops']}",
-                    "traffic": traffic, "algorithmic_flops_per_launch": gemm_flops_per_launch,
-                    "ms_per_launch": g_ms / max(1, g_launch)}
+    roofline = gemm_roofline(H, T, 2 if tdt != torch.float32 else 4, g_launch, g_ms, peaks, traffic_from_profile())
     # memory-bound companions measured in the same region: the packing fused into the first
     # LayerNorm (reads the padded rows once, writes the packed rows and their normalisation)
     # and the pad zeroing; standalone remove / rebuild are timed after the main region
