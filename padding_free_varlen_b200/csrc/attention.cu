@@ -139,12 +139,8 @@ template <typename T, int HD>
 static cudaError_t attn_launch(const void* qkv, void* o, const int32_t* cu, int batch, int max_len, int H,
                                int n_heads, const int32_t* status, cudaStream_t st) {
     constexpr int smem = attn_smem_bytes<HD>();
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(attn_simt_kernel<T, HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    cudaError_t e = prepare_smem((const void*)attn_simt_kernel<T, HD>, smem);
+    if (e != cudaSuccess) return e;
     dim3 grid((max_len + AQB - 1) / AQB, n_heads, batch);
     const float scale = (float)(1.0 / sqrt((double)HD));
     attn_simt_kernel<T, HD><<<grid, 256, smem, st>>>((const T*)qkv, (T*)o, cu, H, scale, status);

@@ -303,22 +303,12 @@ cudaError_t launch_attention_tc(int dtype, const void* qkv, void* o, const int32
     p.timeout_ns = timeout_ns;
     dim3 grid((max_len + ATQ - 1) / ATQ, n_heads, batch);
     if (dtype == ENERGON_BF16) {
-        static bool cfg_b = false;
-        if (!cfg_b) {
-            cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<__nv_bfloat16>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM);
-            if (e != cudaSuccess) return e;
-            cfg_b = true;
-        }
+        cudaError_t e = prepare_smem((const void*)attn_tc_kernel<__nv_bfloat16>, AT_SMEM);
+        if (e != cudaSuccess) return e;
         attn_tc_kernel<__nv_bfloat16><<<grid, 128, AT_SMEM, st>>>(tm, p);
     } else {
-        static bool cfg_h = false;
-        if (!cfg_h) {
-            cudaError_t e =
-                cudaFuncSetAttribute(attn_tc_kernel<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM);
-            if (e != cudaSuccess) return e;
-            cfg_h = true;
-        }
+        cudaError_t e = prepare_smem((const void*)attn_tc_kernel<__half>, AT_SMEM);
+        if (e != cudaSuccess) return e;
         attn_tc_kernel<__half><<<grid, 128, AT_SMEM, st>>>(tm, p);
     }
     return cudaGetLastError();

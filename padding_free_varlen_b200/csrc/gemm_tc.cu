@@ -938,13 +938,8 @@ bool gemm_tc_supported(const GemmArgs& a) {
 template <typename T, int EPI>
 static cudaError_t tc_launch(const CUtensorMap& ta, const CUtensorMap& tb, const TcParams& p, int grid,
                              cudaStream_t st) {
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<T, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             TC_SMEM);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    cudaError_t e = prepare_smem((const void*)gemm_tc_kernel<T, EPI>, TC_SMEM);
+    if (e != cudaSuccess) return e;
     gemm_tc_kernel<T, EPI><<<grid, 256, TC_SMEM, st>>>(ta, tb, p);
     return cudaGetLastError();
 }
@@ -953,16 +948,16 @@ template <typename T, int EPI, int MT>
 static cudaError_t tc2_launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to,
                               const CUtensorMap& tr, const TcParams& p, int pairs, cudaStream_t st) {
     using C = PairCfg<MT>;
-    static int max_pairs = -1;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    if (max_pairs < 0) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_tc2_kernel<T, EPI, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             C::SMEM);
-        if (e != cudaSuccess) return e;
+    const void* kernel = (const void*)gemm_tc2_kernel<T, EPI, MT>;
+    cudaError_t e = prepare_smem(kernel, C::SMEM);
+    if (e != cudaSuccess) return e;
+    // CTA pairs that fit on this device at once (the persistent grid)
+    const int max_pairs = device_cached(kernel, 1, [&] {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(2 * (device_sm_count() / 2));
         cfg.blockDim = dim3(C::THREADS);
@@ -974,8 +969,8 @@ static cudaError_t tc2_launch(const CUtensorMap& ta, const CUtensorMap& tb, cons
             clusters < 1)
             clusters = device_sm_count() / 2;
         (void)cudaGetLastError();
-        max_pairs = clusters;
-    }
+        return clusters;
+    });
     if (pairs > max_pairs) pairs = max_pairs;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * pairs);

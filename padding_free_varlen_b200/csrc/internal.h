@@ -5,7 +5,17 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <functional>
+
 namespace energon {
+
+// Host-side launch facts (a kernel's shared-memory opt-in, its occupancy, the SM count) hold
+// per device: device_cached returns compute() for (current device, key, what), computing it
+// once per triple; thread-safe.
+int device_cached(const void* key, int what, const std::function<int()>& compute);
+// Sets a kernel's dynamic shared-memory limit on the current device once; returns the
+// cudaError_t of that one call on every later call too.
+cudaError_t prepare_smem(const void* kernel, int bytes);
 
 // Offsets: cu[b+1] = cu[b] + lengths[b]; validates lengths into *status (SET).
 cudaError_t launch_offsets(const int32_t* lengths, int batch, int pad_len, int32_t* cu, int32_t* status,

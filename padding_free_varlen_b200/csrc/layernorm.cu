@@ -146,12 +146,14 @@ __global__ void __launch_bounds__(256) ln_vec_kernel(const T* __restrict__ x, co
 // in a single wave of blocks instead of leaving a second wave to start late.
 template <typename K>
 static int resident_blocks(K kernel) {
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, 256, 0) != cudaSuccess || per_sm < 1) {
-        (void)cudaGetLastError();
-        per_sm = 1;
-    }
-    return per_sm * device_sm_count();
+    return device_cached((const void*)kernel, 1, [&] {
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, 256, 0) != cudaSuccess || per_sm < 1) {
+            (void)cudaGetLastError();
+            per_sm = 1;
+        }
+        return per_sm * device_sm_count();
+    });
 }
 
 static int ln_grid(int rows_cap, int resident) {
@@ -171,7 +173,7 @@ static cudaError_t ln_dispatch(const void* x, const void* g, const void* b, void
         switch (vpt) {
 #define LN_CASE(V)                                                                                      \
     case V: {                                                                                           \
-        static const int resident = resident_blocks(ln_vec_kernel<T, V>);                               \
+        const int resident = resident_blocks(ln_vec_kernel<T, V>);                                      \
         ln_vec_kernel<T, V><<<ln_grid(rows_cap, resident), 256, 0, st>>>(xp, gp, bp, yp, d_rows, rows_cap, H, \
                                                                          eps, status, gth);             \
         break;                                                                                          \
@@ -180,7 +182,7 @@ static cudaError_t ln_dispatch(const void* x, const void* g, const void* b, void
 #undef LN_CASE
         }
     } else {
-        static const int resident = resident_blocks(ln_generic_kernel<T>);
+        const int resident = resident_blocks(ln_generic_kernel<T>);
         ln_generic_kernel<T><<<ln_grid(rows_cap, resident), 256, 0, st>>>(xp, gp, bp, yp, d_rows, rows_cap, H, eps,
                                                                          status, gth);
     }
@@ -192,7 +194,7 @@ template <>
 cudaError_t ln_dispatch<float>(const void* x, const void* g, const void* b, void* y, const int32_t* d_rows,
                                int rows_cap, int H, float eps, const int32_t* status, const LnGather& gth,
                                cudaStream_t st) {
-    static const int resident = resident_blocks(ln_generic_kernel<float>);
+    const int resident = resident_blocks(ln_generic_kernel<float>);
     ln_generic_kernel<float><<<ln_grid(rows_cap, resident), 256, 0, st>>>(
         (const float*)x, (const float*)g, (const float*)b, (float*)y, d_rows, rows_cap, H, eps, status, gth);
     return cudaGetLastError();

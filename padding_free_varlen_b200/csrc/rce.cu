@@ -9,20 +9,53 @@
 // remove/rebuild move 16-byte vectors when the row size and both base
 // pointers allow it, one warp per row, grid-stride over rows; the grid is a
 // multiple of the SM count so every SM keeps several rows in flight.
+#include <map>
+#include <mutex>
+#include <tuple>
+
 #include "common.cuh"
 #include "internal.h"
 
 namespace energon {
 
-int device_sm_count() {
-    static int sms = 0;
-    if (sms == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (sms <= 0) sms = 148;
+int device_cached(const void* key, int what, const std::function<int()>& compute) {
+    static std::mutex mu;
+    static std::map<std::tuple<int, const void*, int>, int> cache;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        (void)cudaGetLastError();
+        dev = -1;
     }
-    return sms;
+    const auto k = std::make_tuple(dev, key, what);
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        auto it = cache.find(k);
+        if (it != cache.end()) return it->second;
+    }
+    // Computed without the lock (compute may itself ask the cache, e.g. for the SM count);
+    // two threads may both compute it once, the first stored value wins.
+    const int v = compute();
+    std::lock_guard<std::mutex> lock(mu);
+    return cache.emplace(k, v).first->second;
+}
+
+cudaError_t prepare_smem(const void* kernel, int bytes) {
+    return (cudaError_t)device_cached(kernel, 0, [&] {
+        return (int)cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    });
+}
+
+int device_sm_count() {
+    static const int tag = 0;
+    return device_cached(&tag, 0, [] {
+        int dev = 0, sms = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
+            (void)cudaGetLastError();
+            sms = 148;
+        }
+        return sms;
+    });
 }
 
 // ------------------------------------------------------------------ offsets
