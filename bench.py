@@ -184,7 +184,7 @@ def run_reference(args, dist: Dist):
     lengths, S = wl.lengths(), wl.padded_len()
     T = int(lengths.sum())
     x = wl.x_padded()
-    tokens = args.cpu_tokens or 2
+    tokens = args.cpu_tokens or 1
     n = args.warmup + args.steps
     seqs = [i % wl.batch for i in range(n)]
     ps = [int(min(tokens, lengths[b])) for b in seqs]
