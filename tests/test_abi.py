@@ -128,3 +128,37 @@ def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     monkeypatch.setattr(capi, "LIB_PATH", str(tmp_path / "absent.so"))
     with pytest.raises(RuntimeError, match="missing"):
         capi.load()
+
+
+def test_header_is_c_and_struct_layouts_match_the_binding(tmp_path):
+    """The header compiles as C11, and every struct has the size and field offsets the
+    ctypes binding assumes (gcc prints them; no GPU needed)."""
+    import ctypes
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    structs = {
+        "energon_layer_weights": (capi.energon_layer_weights, list(capi.WEIGHT_FIELDS)),
+        "energon_layer_config": (capi.energon_layer_config, ["hidden", "n_heads", "ffn", "dtype", "ln_eps",
+                                                             "gelu_tanh"]),
+        "energon_trace_entry": (capi.energon_trace_entry, ["name", "launches", "total_ms"]),
+        "energon_request": (capi.energon_request, ["length", "arrival_s"]),
+    }
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "energon_rce.h"', "int main(void) {"]
+    for name, (_, fields) in structs.items():
+        lines.append(f'    printf("{name} size %zu\\n", sizeof({name}));')
+        for f in fields:
+            lines.append(f'    printf("{name} {f} %zu\\n", offsetof({name}, {f}));')
+    lines += ["    return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    include = os.path.join(ROOT, "include")
+    subprocess.run(["gcc", "-std=c11", "-Wall", "-Werror", "-I", include, str(src), "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split("\n")
+    got = {tuple(l.split()[:2]): int(l.split()[2]) for l in out if l.strip()}
+    for name, (cls, fields) in structs.items():
+        assert got[(name, "size")] == ctypes.sizeof(cls), name
+        for f in fields:
+            assert got[(name, f)] == getattr(cls, f).offset, (name, f)
