@@ -6,6 +6,7 @@ import os
 import random
 
 import pytest
+from hypothesis import given, settings, strategies as hs
 
 from padding_free_varlen_b200 import capi, synth
 
@@ -66,3 +67,23 @@ def test_plan_rejects_bad_arguments():
         assert e.value.code == capi.ENERGON_ERR_INVALID_ARGUMENT
     with pytest.raises(capi.EnergonError):
         capi.energon_sched_fifo([0.0, 1.0], 0)
+
+
+@settings(max_examples=150, deadline=None)
+@given(data=hs.data())
+def test_plan_matches_oracle_on_arbitrary_queues(data):
+    """Random queues (ties in length and arrival included) and random positive cost tables,
+    monotone or not: the C++ runtime and the oracle take the same decisions."""
+    n = data.draw(hs.integers(0, 40))
+    max_b = data.draw(hs.integers(1, 8))
+    max_s = data.draw(hs.integers(1, 12))
+    lengths = data.draw(hs.lists(hs.integers(1, max_s), min_size=n, max_size=n))
+    arrivals = data.draw(hs.lists(hs.sampled_from([0.0, 0.25, 0.5, 1.0, 2.0]), min_size=n, max_size=n))
+    table = data.draw(hs.lists(hs.lists(hs.floats(0.01, 100.0), min_size=max_s, max_size=max_s),
+                               min_size=max_b, max_size=max_b))
+    now = data.draw(hs.sampled_from([2.0, 3.5, 10.0]))
+    age = data.draw(hs.sampled_from([0.1, 1.0, 7.0]))
+    got = capi.energon_sched_plan(lengths, arrivals, now, max_b, table, age)
+    ref = oracle_sched.plan(lengths, arrivals, now, max_b, table, age)
+    assert got == (list(ref[0]), list(ref[1]))
+    assert capi.energon_sched_fifo(arrivals, max_b) == oracle_sched.fifo(arrivals, max_b)
