@@ -245,14 +245,37 @@ def gemm_roofline(H: int, T: int, elem_bytes: int, launches: int, ms_total: floa
         return {"bound": "hbm", "kernel": "gemm_tc (tcgen05, 4 shapes per layer), weight streaming",
                 "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"] if achieved else None,
+                "frac_of_datasheet": achieved / DATASHEET_HBM_GBS if achieved else None,
                 "peak_note": f"{peaks['source']} HBM copy rate", "traffic": None,
                 "algorithmic_bytes_per_launch": weight_bytes_per_launch, "ms_per_launch": ms_per_launch}
     achieved = flops_per_launch * launches / (ms_total / 1e3) / 1e12 if ms_total > 0 else None
     return {"bound": "tensor", "kernel": "gemm_tc (tcgen05, 4 shapes per layer)",
             "achieved": achieved, "peak": peaks["tflops_sustained"], "unit": "TFLOP/s",
             "frac": achieved / peaks["tflops_sustained"] if achieved else None,
+            "frac_of_burst": achieved / peaks["tflops"] if achieved else None,
+            "frac_of_datasheet": achieved / DATASHEET_TFLOPS if achieved else None,
             "peak_note": f"{peaks['source']} bf16 sustained (fp16 assumed at the bf16 rate); burst {peaks['tflops']}",
             "traffic": traffic, "algorithmic_flops_per_launch": flops_per_launch, "ms_per_launch": ms_per_launch}
+
+
+DATASHEET_TFLOPS = 2250.0    # dense fp16 / bf16, for context
+DATASHEET_HBM_GBS = 8000.0
+
+
+def step_roofline(H: int, n_layers: int, lengths, elem_bytes: int, ms_per_step: float, peaks: dict) -> dict:
+    """The whole step against its roofline: t_roof = max(algorithmic flop / sustained tensor
+    peak, weight bytes / HBM rate), flop = per layer 24 H^2 T for the four GEMMs plus 4 H per
+    visible key-query pair for QK^T and PV (sum over sequences of L (L + 1) / 2 pairs)."""
+    T = int(sum(int(v) for v in lengths))
+    pairs = sum(int(v) * (int(v) + 1) // 2 for v in lengths)
+    flop = n_layers * (24 * H * H * T + 4 * H * pairs)
+    weight_bytes = n_layers * 12 * H * H * elem_bytes
+    t_flop = flop / (peaks["tflops_sustained"] * 1e12) * 1e3
+    t_bytes = weight_bytes / (peaks["hbm_gbs"] * 1e9) * 1e3
+    t_roof = max(t_flop, t_bytes)
+    return {"algorithmic_flop": flop, "weight_bytes": weight_bytes, "t_roof_ms": t_roof,
+            "bound": "tensor" if t_flop >= t_bytes else "hbm", "ms_per_step": ms_per_step,
+            "frac": t_roof / ms_per_step if ms_per_step > 0 else None}
 
 
 def run_energon(args, dist: Dist):
@@ -376,6 +399,7 @@ def run_energon(args, dist: Dist):
     per_kernel = {k: {"launches": v[0], "ms_per_step": v[1] / args.steps,
                       "share": v[1] / max(1e-9, sum(x[1] for x in trace.values()))} for k, v in trace.items()}
     roofline = gemm_roofline(H, T, 2 if tdt != torch.float32 else 4, g_launch, g_ms, peaks, traffic_from_profile())
+    whole_step = step_roofline(H, L, lengths, 2 if tdt != torch.float32 else 4, ms / args.steps, peaks)
     # memory-bound companions measured in the same region: the packing fused into the first
     # LayerNorm (reads the padded rows once, writes the packed rows and their normalisation)
     # and the pad zeroing; standalone remove / rebuild are timed after the main region
@@ -516,7 +540,8 @@ def run_energon(args, dist: Dist):
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f16" if tdt == torch.float16 else str(tdt).replace("torch.", ""),
             "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights)",
-            "config": config_of(wl, S, T, dist.world), "roofline": roofline, "roofline_memory_kernels": aux,
+            "config": config_of(wl, S, T, dist.world), "roofline": roofline, "step_roofline": whole_step,
+            "roofline_memory_kernels": aux,
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clk,
             "padded_path": padded, "transpose_forms": transpose, "dynamic_batching": batching,
             "kernels": per_kernel, "setup_s": setup_s}

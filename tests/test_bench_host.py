@@ -43,3 +43,24 @@ def test_bound_switches_at_the_ridge():
     assert bench.gemm_roofline(H, below, 2, 4, 1.0, PEAKS, None)["bound"] == "hbm"
     assert bench.gemm_roofline(H, above, 2, 4, 1.0, PEAKS, None)["bound"] == "tensor"
     assert bench.gemm_roofline(H, 100, 2, 0, 0.0, PEAKS, None)["achieved"] is None
+
+
+def test_step_roofline_matches_the_worked_figures():
+    # 12 layers, batch 32 of length 128 at H 12288: 1.783e14 flop; 126.4 ms at 1410 TFLOP/s
+    r = bench.step_roofline(12288, 12, [128] * 32, 2, 148.5, PEAKS)
+    assert r["algorithmic_flop"] == 12 * (24 * 12288 ** 2 * 4096 + 4 * 12288 * 32 * 128 * 129 // 2)
+    assert r["algorithmic_flop"] == pytest.approx(1.783e14, rel=1e-3)
+    assert r["bound"] == "tensor" and r["t_roof_ms"] == pytest.approx(126.4, rel=2e-3)
+    assert r["frac"] == pytest.approx(r["t_roof_ms"] / 148.5)
+    # one layer at T = 32: the weights (3.62 GB) bound it, 0.562 ms at 6443 GB/s
+    r = bench.step_roofline(12288, 1, [32], 2, 0.727, PEAKS)
+    assert r["bound"] == "hbm" and r["weight_bytes"] == 12 * 12288 ** 2 * 2
+    assert r["t_roof_ms"] == pytest.approx(0.5624, rel=2e-3)
+
+
+def test_fractions_of_burst_and_datasheet():
+    r = bench.gemm_roofline(12288, 4096, 2, 480, 1430.0, PEAKS, None)
+    assert r["frac_of_burst"] == pytest.approx(r["achieved"] / 1671.8)
+    assert r["frac_of_datasheet"] == pytest.approx(r["achieved"] / 2250.0)
+    r = bench.gemm_roofline(12288, 32, 2, 40, 6.4, PEAKS, None)
+    assert r["frac_of_datasheet"] == pytest.approx(r["achieved"] / 8000.0)
