@@ -165,7 +165,9 @@ typedef struct {
  *   batch * pad_len <= 128, else 0 bytes        - used by both calls
  *   x [R, H], cu [batch + 1] int32, cu_pad [batch + 1] int32 - stack only
  * After a call completes, the regions hold that call's (last layer's)
- * intermediates for the first T rows, which makes every step inspectable.
+ * intermediates for the first T rows, which makes every step inspectable
+ * (the stack with remove_padding = 2 reuses o and qkv for the packed input and
+ * output of the last MLP).
  */
 ENERGON_API size_t energon_workspace_bytes(const energon_layer_config* cfg, int batch, int pad_len);
 
@@ -192,7 +194,11 @@ ENERGON_API int energon_layer_forward(const energon_layer_config* cfg, const ene
 
 /*
  * The whole hot path: offsets -> transpose_padding_remove -> n_layers decoder
- * layers on packed tokens -> transpose_padding_rebuild.
+ * layers on packed tokens -> transpose_padding_rebuild.  With remove_padding = 1
+ * the remove is fused into the first LayerNorm (it gathers the valid rows) and
+ * the rebuild into the last FFN2 GEMM's epilogue (it stores each row at its
+ * padded position; the pad rows are zeroed by a separate launch) whenever that
+ * GEMM runs on the CTA-pair kernel, i.e. more than 128 rows of capacity.
  *   layers        host array of n_layers weight tables
  *   padded_in     [batch, pad_len, H] device; pad positions may hold anything
  *   lengths       [batch] int32, device
@@ -231,7 +237,8 @@ ENERGON_API void energon_set_wait_timeout_us(uint32_t timeout_us);
  * energon_trace_stop, every kernel that energon_layer_forward and
  * energon_stack_forward launch is bracketed by two CUDA events on the call's
  * stream.  energon_trace_stop synchronises those events and writes, per kernel
- * name ("gemm_qkv", "attention", "layernorm", "remove_padding", ...), the number
+ * name ("gemm_qkv", "attention", "layernorm", "layernorm_remove", "zero_pads",
+ * "gemm_ffn2_rebuild", "remove_padding", ...), the number
  * of launches and their summed device time in milliseconds.  Recording adds a
  * pair of event records per launch and nothing else.  Process-wide; not
  * thread-safe.  *n_entries receives the number of names (at most capacity are
