@@ -69,3 +69,10 @@ def test_reference_arm_two_ranks_rank0_prints():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
+    # the keys every bench line carries
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+              "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert k in d, k
+    assert d["steps"] == 2 and d["warmup"] == 1 and d["higher_is_better"] is True and d["scaling"] == "weak"
+    assert d["config"]["workload"] == "tiny" and d["e2e"]["unit"] == d["unit"]
+    assert {"value", "unit", "cores", "kind", "sample"} <= set(d["cpu_baseline"])
