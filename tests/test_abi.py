@@ -162,3 +162,8 @@ def test_header_is_c_and_struct_layouts_match_the_binding(tmp_path):
         assert got[(name, "size")] == ctypes.sizeof(cls), name
         for f in fields:
             assert got[(name, f)] == getattr(cls, f).offset, (name, f)
+
+
+def test_every_export_has_a_binding_of_the_same_name():
+    missing = [n for n in capi.EXPORTED if not callable(getattr(capi, n, None))]
+    assert not missing, missing
