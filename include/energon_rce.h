@@ -228,6 +228,15 @@ ENERGON_API int energon_stack_forward(const energon_layer_config* cfg, const ene
  */
 ENERGON_API int energon_selftest_bounded_wait(int32_t* d_status, uint32_t timeout_us, void* stream);
 
+/*
+ * Build check (diagnostic; no counterpart in the pages): the binary version that
+ * the CUDA runtime reports for the library's kernels on the current device
+ * (cudaFuncGetAttributes, major * 10 + minor: 100 for the sm_100a build).
+ * Needs a device; launches nothing.  Errors: NULL -> ENERGON_ERR_INVALID_ARGUMENT;
+ * no device or no kernel image for it -> ENERGON_ERR_CUDA.
+ */
+ENERGON_API int energon_kernel_binary_version(int* version);
+
 /* Upper limit, in microseconds, of every bounded wait inside the kernels
  * (default 2,000,000).  Process-wide. */
 ENERGON_API void energon_set_wait_timeout_us(uint32_t timeout_us);
@@ -269,8 +278,11 @@ ENERGON_API int energon_trace_stop(energon_trace_entry* entries, int capacity, i
  * with ENERGON_ERR_INVALID_ARGUMENT before anything is launched.  The call
  * allocates nothing.  The first call on a device looks up the array's device
  * address (cudaGetSymbolAddress), so make that first call before any stream
- * capture.  All calls on a device share the array: calls that may overlap on
- * the GPU (unordered streams) race; calls ordered on one stream do not.
+ * capture.  The address is kept per device and per context: cudaDeviceReset
+ * unloads the library's device image, and the first call after it looks the
+ * address up again in the new context (make that call before any capture too).
+ * All calls on a device share the array: calls that may overlap on the GPU
+ * (unordered streams) race; calls ordered on one stream do not.
  */
 #define ENERGON_NOALLOC_MAX_BATCH 16384
 ENERGON_API int energon_rce_remove_padding_noalloc(const void* padded, const int32_t* lengths, int batch,

@@ -37,7 +37,7 @@ EXPORTED = ("energon_rce_offsets", "energon_rce_remove_padding", "energon_rce_re
             "energon_selftest_bounded_wait", "energon_set_wait_timeout_us", "energon_last_error",
             "energon_trace_start", "energon_trace_stop", "energon_rce_remove_padding_noalloc",
             "energon_rce_transpose_padding_rebuild", "energon_rce_transpose_padding_remove",
-            "energon_sched_plan", "energon_sched_fifo")
+            "energon_sched_plan", "energon_sched_fifo", "energon_kernel_binary_version")
 ENERGON_NOALLOC_MAX_BATCH = 16384
 WEIGHT_FIELDS = ("ln1_g", "ln1_b", "w_qkv", "b_qkv", "w_o", "b_o",
                  "ln2_g", "ln2_b", "w_1", "b_1", "w_2", "b_2")
@@ -88,6 +88,7 @@ def load() -> ctypes.CDLL:
             "energon_layer_forward": ([cfgp, wp, vp, vp, ci, ci, vp, vp, vp, sz, vp], ci),
             "energon_stack_forward": ([cfgp, wp, ci, vp, vp, ci, ci, ci, vp, vp, vp, sz, vp], ci),
             "energon_selftest_bounded_wait": ([vp, u32, vp], ci),
+            "energon_kernel_binary_version": ([ctypes.POINTER(ci)], ci),
             "energon_set_wait_timeout_us": ([u32], None),
             "energon_last_error": ([], ctypes.c_char_p),
             "energon_trace_start": ([], ci),
@@ -213,6 +214,12 @@ def energon_stack_forward(cfg, layers, n_layers, padded_in, lengths, batch, pad_
 def energon_selftest_bounded_wait(d_status, timeout_us, stream=None) -> None:
     _check(load().energon_selftest_bounded_wait(_dev(d_status, "d_status"), int(timeout_us), _stream(stream)),
            "energon_selftest_bounded_wait")
+
+
+def energon_kernel_binary_version() -> int:
+    v = ctypes.c_int(0)
+    _check(load().energon_kernel_binary_version(ctypes.byref(v)), "energon_kernel_binary_version")
+    return v.value
 
 
 def energon_trace_start() -> None:

@@ -189,7 +189,9 @@ int run_gemm(GemmArgs& g, cudaStream_t st, const char* what) {
         }
         return ENERGON_OK;
     }
-    CK(traced(what, st, [&] { return launch_gemm_simt(g, st); }), what);
+    // Shapes the tensor-core kernel does not take (fp32, or 16-bit N / K off its tile
+    // multiples) run on the CUDA-core kernel; the trace names it apart.
+    CK(traced("gemm_simt", st, [&] { return launch_gemm_simt(g, st); }), what);
     return ENERGON_OK;
 }
 
@@ -541,6 +543,13 @@ int energon_trace_stop(energon_trace_entry* entries, int capacity, int* n_entrie
     g_event_used = 0;
     if (n_entries) *n_entries = (int)agg.size();
     for (int i = 0; entries && i < capacity && i < (int)agg.size(); ++i) entries[i] = agg[i];
+    return ENERGON_OK;
+}
+
+int energon_kernel_binary_version(int* version) {
+    g_last_error.clear();
+    if (!version) return fail(ENERGON_ERR_INVALID_ARGUMENT, "kernel_binary_version: NULL pointer");
+    CK(kernel_binary_version(version), "kernel_binary_version");
     return ENERGON_OK;
 }
 

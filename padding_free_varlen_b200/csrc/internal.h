@@ -97,6 +97,9 @@ bool attention_tc_supported(int dtype, int H, int n_heads, const void* qkv, cons
 cudaError_t launch_attention_tc(int dtype, const void* qkv, void* o, const int32_t* cu, int batch, int max_len, int H,
                                 int n_heads, int qkv_rows, int32_t* status, uint64_t timeout_ns, cudaStream_t st);
 
+// The binary version (major * 10 + minor) the runtime reports for the library's kernels.
+cudaError_t kernel_binary_version(int* version);
+
 // Self-test kernel of the bounded wait.
 cudaError_t launch_wait_selftest(int32_t* status, uint64_t timeout_ns, cudaStream_t st);
 

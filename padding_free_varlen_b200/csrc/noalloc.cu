@@ -32,21 +32,48 @@ namespace {
 constexpr int kMaxDevices = 128;
 std::mutex g_addr_mu;
 int32_t* g_addr[kMaxDevices] = {};
+CUcontext g_addr_ctx[kMaxDevices] = {};
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+// The driver's cuCtxGetCurrent, found through the runtime (the library does not link
+// the driver library directly); null if it cannot be found.
+CtxGetCurrentFn ctx_get_current() {
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+    });
+    return fn;
+}
 
 // Device address of the scratch array on the current device.  In host code the
 // array's name is only a host-side stand-in, so the address is looked up once
-// per device (with that device current) and reused.
+// per device (with that device current) and reused.  The lookup is keyed by the
+// device's current context as well: cudaDeviceReset destroys the context and the
+// library's device image with it, and the first call after it (in the new
+// context) looks the address up again instead of using the old one.
 cudaError_t scratch_address(int32_t** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    CtxGetCurrentFn get = ctx_get_current();
+    if (get == nullptr) return cudaErrorInitializationError;
+    CUcontext ctx = nullptr;
+    if (get(&ctx) != CUDA_SUCCESS) ctx = nullptr;  // null until the runtime has set up this device
     std::lock_guard<std::mutex> lock(g_addr_mu);
-    if (g_addr[dev] == nullptr) {
+    if (g_addr[dev] == nullptr || ctx == nullptr || g_addr_ctx[dev] != ctx) {
         void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_offsets);
+        e = cudaGetSymbolAddress(&p, g_noalloc_offsets);  // sets up the primary context if needed
         if (e != cudaSuccess) return e;
+        if (get(&ctx) != CUDA_SUCCESS) ctx = nullptr;
         g_addr[dev] = static_cast<int32_t*>(p);
+        g_addr_ctx[dev] = ctx;
     }
     *out = g_addr[dev];
     return cudaSuccess;

@@ -107,6 +107,13 @@ __global__ void __launch_bounds__(1024) offsets_kernel(const int32_t* __restrict
     if (tid == 0) *status = bad ? ENERGON_DEVICE_BAD_LENGTH : ENERGON_DEVICE_OK;
 }
 
+cudaError_t kernel_binary_version(int* version) {
+    cudaFuncAttributes a;
+    cudaError_t e = cudaFuncGetAttributes(&a, offsets_kernel);
+    if (e == cudaSuccess) *version = a.binaryVersion;
+    return e;
+}
+
 cudaError_t launch_offsets(const int32_t* lengths, int batch, int pad_len, int32_t* cu, int32_t* status,
                            cudaStream_t st) {
     int threads = batch >= 1024 ? 1024 : ((batch + 31) / 32) * 32;

@@ -130,3 +130,8 @@ def test_remove_rebuild_workload_full_size(oracle_lib, synth_mod):
     capi.energon_rce_remove_padding(d_x, d_cu_full, B, S, H, 2, pk)
     torch.cuda.synchronize()
     assert torch.equal(pk.view(torch.int16), d_x.view(B * S, H).view(torch.int16))
+
+
+def test_kernels_are_sm100a_binaries():
+    """The runtime reports binary version 100 (sm_100a) for the library's kernels."""
+    assert capi.energon_kernel_binary_version() == 100
