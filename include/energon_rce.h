@@ -158,16 +158,22 @@ typedef struct {
  *
  * Layout (part of the ABI; each region starts on a 1024-byte boundary, e =
  * element bytes, R = batch * pad_len rounded up to a multiple of 256):
- *   a [R, H]   LayerNorm output (after a layer call: the second LayerNorm's)
- *   qkv [R, 3H], o [R, H] (attention output), x1 [R, H] (residual after
- *   attention), f [R, F] (GELU output)      - used by both calls
- *   p32: fp32 split-K partial sums, 4 * 128 * max(3H, F) floats when
- *   batch * pad_len <= 128, else 0 bytes        - used by both calls
+ *   a [R, H]      GEMM operand of the LayerNorms: u = x * ln1_g for the folded
+ *                 first LayerNorm, then the second LayerNorm's output
+ *   qkv [R, 3H]   Q | K | V (for 16-bit types, Q and K are the high halves)
+ *   qk_lo [R, 2H] low halves of Q | K (16-bit types; 0 bytes for fp32)
+ *   o [R, H]      attention output
+ *   x1 [R, H]     fp32: the residual after attention
+ *   f [R, F]      GELU output
+ *   p32           fp32 split-K partial sums, 4 * 128 * max(3H, F) floats when
+ *                 batch * pad_len <= 128, else 0 bytes
+ *   stats [R]     float2 per row: (rstd, mean * rstd) of the first LayerNorm
+ *   fold [6H]     fp32: c = W_qkv ln1_g [3H], then d = b_qkv + W_qkv ln1_b [3H]
  *   x [R, H], cu [batch + 1] int32, cu_pad [batch + 1] int32 - stack only
  * After a call completes, the regions hold that call's (last layer's)
  * intermediates for the first T rows, which makes every step inspectable
- * (the stack with remove_padding = 2 reuses o and qkv for the packed input and
- * output of the last MLP).
+ * (the stack with remove_padding = 2 reuses qkv and o for the packed fp32
+ * input and the packed output of the last MLP).
  */
 ENERGON_API size_t energon_workspace_bytes(const energon_layer_config* cfg, int batch, int pad_len);
 
@@ -182,10 +188,15 @@ ENERGON_API size_t energon_workspace_bytes(const energon_layer_config* cfg, int 
  *   max_len: the largest sequence length (pad_len); sizes the launch grids.
  *   d_status: optional device status word (NULL allowed); kernels skip work when
  *   it is nonzero and OR ENERGON_DEVICE_TIMEOUT into it if a bounded wait expires.
- * LayerNorm statistics, accumulation and softmax are fp32; every kernel
- * boundary rounds to the storage dtype.  fp16 / bf16 use the tcgen05 tensor-core
- * GEMM when H % 256 == 0 and F % 256 == 0; fp32 uses CUDA-core kernels.
- * head_dim must be 64 or 128.
+ * LayerNorm statistics, accumulation and softmax are fp32.  The first LayerNorm
+ * is folded into the QKV GEMM (its operand is the layer input times ln1_g, one
+ * rounding, exact when ln1_g is 1; the epilogue applies the row statistics), Q
+ * and K are kept as two 16-bit terms for the attention scores, and the residual
+ * after attention stays in fp32; the other kernel boundaries (V, the attention
+ * output, the second LayerNorm, the GELU output, y) round to the storage dtype.
+ * fp16 / bf16 use the tcgen05 tensor-core GEMM when H % 256 == 0 and
+ * F % 256 == 0 (other shapes run the CUDA-core GEMM, traced as "gemm_simt");
+ * fp32 uses CUDA-core kernels.  head_dim must be 64 or 128.
  */
 ENERGON_API int energon_layer_forward(const energon_layer_config* cfg, const energon_layer_weights* w,
                           const void* x_packed, const int32_t* cu_seqlens, int batch, int max_len,

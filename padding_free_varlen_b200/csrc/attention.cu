@@ -3,7 +3,8 @@
 // For sequence b (packed rows cu[b] .. cu[b+1]-1), head j and position s:
 //     o_j(s) = sum_{t <= s} softmax_t(q_j(s) . k_j(t) / sqrt(d)) v_j(t)
 // with q, k, v read from the fused projection qkv [rows, 3H] (columns Q | K | V,
-// head-major inside each).  Keys never cross a sequence boundary, so padding
+// head-major inside each); when the low halves qk_lo [rows, 2H] are given, q and
+// k are hi + lo.  Keys never cross a sequence boundary, so padding
 // and other sequences never enter: this is what lets the layer run on the
 // packed tokens only (EnergonAI README, "Scaling Ability": redundant
 // computation elimination in the GPT-3 layers).
@@ -34,9 +35,9 @@ constexpr int attn_smem_bytes() {
 }
 
 template <typename T, int HD>
-__global__ void __launch_bounds__(256) attn_simt_kernel(const T* __restrict__ qkv, T* __restrict__ out,
-                                                        const int32_t* __restrict__ cu, int H, float scale,
-                                                        const int32_t* status) {
+__global__ void __launch_bounds__(256) attn_simt_kernel(const T* __restrict__ qkv, const T* __restrict__ qk_lo,
+                                                        T* __restrict__ out, const int32_t* __restrict__ cu, int H,
+                                                        float scale, const int32_t* status) {
     constexpr int QPW = AQB / ANW;  // queries per warp
     constexpr int DPL = HD / 32;    // output dims per lane
     extern __shared__ float smem[];
@@ -53,9 +54,16 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(const T* __restrict__ qk
     const int64_t ld = 3 * (int64_t)H;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
+    const int64_t ldl = 2 * (int64_t)H;  // qk_lo: the low halves of Q | K (q = hi + lo)
     for (int e = tid; e < AQB * HD; e += blockDim.x) {
         const int r = e / HD, d = e % HD;
-        Qs[e] = (q0 + r < q_end) ? to_f(qkv[(int64_t)(start + q0 + r) * ld + (int64_t)j * HD + d]) : 0.0f;
+        float qv = 0.0f;
+        if (q0 + r < q_end) {
+            const int64_t row = start + q0 + r;
+            qv = to_f(qkv[row * ld + (int64_t)j * HD + d]);
+            if (qk_lo) qv += to_f(qk_lo[row * ldl + (int64_t)j * HD + d]);
+        }
+        Qs[e] = qv;
     }
 
     float m[QPW], l[QPW], acc[QPW][DPL];
@@ -74,8 +82,10 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(const T* __restrict__ qk
             const int t = e / HD, d = e % HD;
             float kv = 0.0f, vv = 0.0f;
             if (t < kn) {
-                const int64_t row = (int64_t)(start + kc0 + t) * ld + (int64_t)j * HD + d;
+                const int64_t tok = start + kc0 + t;
+                const int64_t row = tok * ld + (int64_t)j * HD + d;
                 kv = to_f(qkv[row + H]);
+                if (qk_lo) kv += to_f(qk_lo[tok * ldl + H + (int64_t)j * HD + d]);
                 vv = to_f(qkv[row + 2 * (int64_t)H]);
             }
             Ks[t * (HD + 1) + d] = kv;
@@ -136,27 +146,29 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(const T* __restrict__ qk
 }
 
 template <typename T, int HD>
-static cudaError_t attn_launch(const void* qkv, void* o, const int32_t* cu, int batch, int max_len, int H,
-                               int n_heads, const int32_t* status, cudaStream_t st) {
+static cudaError_t attn_launch(const void* qkv, const void* qk_lo, void* o, const int32_t* cu, int batch,
+                               int max_len, int H, int n_heads, const int32_t* status, cudaStream_t st) {
     constexpr int smem = attn_smem_bytes<HD>();
     cudaError_t e = prepare_smem((const void*)attn_simt_kernel<T, HD>, smem);
     if (e != cudaSuccess) return e;
     dim3 grid((max_len + AQB - 1) / AQB, n_heads, batch);
     const float scale = (float)(1.0 / sqrt((double)HD));
-    attn_simt_kernel<T, HD><<<grid, 256, smem, st>>>((const T*)qkv, (T*)o, cu, H, scale, status);
+    attn_simt_kernel<T, HD><<<grid, 256, smem, st>>>((const T*)qkv, (const T*)qk_lo, (T*)o, cu, H, scale, status);
     return cudaGetLastError();
 }
 
-cudaError_t launch_attention(int dtype, const void* qkv, void* o, const int32_t* cu, int batch, int max_len, int H,
-                             int n_heads, int qkv_rows, int32_t* status, uint64_t timeout_ns, cudaStream_t st) {
+cudaError_t launch_attention(int dtype, const void* qkv, const void* qk_lo, void* o, const int32_t* cu, int batch,
+                             int max_len, int H, int n_heads, int qkv_rows, int32_t* status, uint64_t timeout_ns,
+                             cudaStream_t st) {
     if (batch <= 0 || max_len <= 0) return cudaSuccess;
-    if (attention_tc_supported(dtype, H, n_heads, qkv, o, qkv_rows))
-        return launch_attention_tc(dtype, qkv, o, cu, batch, max_len, H, n_heads, qkv_rows, status, timeout_ns, st);
+    if (attention_tc_supported(dtype, H, n_heads, qkv, qk_lo, o, qkv_rows))
+        return launch_attention_tc(dtype, qkv, qk_lo, o, cu, batch, max_len, H, n_heads, qkv_rows, status, timeout_ns,
+                                   st);
     const int hd = H / n_heads;
     if (hd != 64 && hd != 128) return cudaErrorInvalidValue;
 #define ATTN_CASE(T)                                                                                     \
-    return hd == 64 ? attn_launch<T, 64>(qkv, o, cu, batch, max_len, H, n_heads, status, st)            \
-                    : attn_launch<T, 128>(qkv, o, cu, batch, max_len, H, n_heads, status, st);
+    return hd == 64 ? attn_launch<T, 64>(qkv, qk_lo, o, cu, batch, max_len, H, n_heads, status, st)     \
+                    : attn_launch<T, 128>(qkv, qk_lo, o, cu, batch, max_len, H, n_heads, status, st);
     switch (dtype) {
     case ENERGON_F32: ATTN_CASE(float)
     case ENERGON_F16: ATTN_CASE(__half)

@@ -33,7 +33,9 @@ constexpr int ATQ = 128;                // queries per CTA
 constexpr int ATK = 128;                // keys per block
 constexpr int AHD = 128;                // head dim
 constexpr int ATILE = 128 * 64 * 2;     // 128 rows x 64 columns of 16-bit = 16 KiB, one swizzle block column
-constexpr int AT_SMEM = 6 * ATILE + 1024 + 128;
+// Q, K, V (and with the low halves of Q and K, two more) tiles of 128 x 128.
+template <bool LO>
+constexpr int at_smem() { return (LO ? 10 : 6) * ATILE + 1024 + 128; }
 constexpr uint32_t AT_TMEM_COLS = 256;  // S: 0..127, O: 128..255
 }  // namespace
 
@@ -53,14 +55,19 @@ __device__ __forceinline__ bool block_wait(uint64_t* bar, uint32_t parity, uint6
     return __syncthreads_and(ok) != 0;
 }
 
-template <typename T>
-__global__ void __launch_bounds__(128) attn_tc_kernel(const __grid_constant__ CUtensorMap tm, const AttnTcParams p) {
+// LO: the low halves of Q and K (tensor map tml over qk_lo [rows, 2H]) enter the scores,
+// S = Qh Kh^T + Qh Kl^T + Ql Kh^T (the Ql Kl^T term is below fp32 resolution).
+template <typename T, bool LO>
+__global__ void __launch_bounds__(128) attn_tc_kernel(const __grid_constant__ CUtensorMap tm,
+                                                      const __grid_constant__ CUtensorMap tml, const AttnTcParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sQ = base;              // Q: head dims 0..63 | 64..127
     uint8_t* sK = base + 2 * ATILE;  // K: head dims 0..63 | 64..127; then P: keys 0..63 | 64..127
     uint8_t* sV = base + 4 * ATILE;  // V: head dims 0..63 | 64..127, one row per key
-    uint64_t* bars = reinterpret_cast<uint64_t*>(base + 6 * ATILE);
+    uint8_t* sQl = base + 6 * ATILE; // low halves of Q and K (LO only)
+    uint8_t* sKl = base + 8 * ATILE;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(base + (LO ? 10 : 6) * ATILE);
     uint64_t* bar_q = bars;
     uint64_t* bar_kv = bars + 1;
     uint64_t* bar_mma = bars + 2;
@@ -94,16 +101,27 @@ __global__ void __launch_bounds__(128) attn_tc_kernel(const __grid_constant__ CU
     const int colQ = j * AHD, colK = p.H + j * AHD, colV = 2 * p.H + j * AHD;
     bool q_pending = false, kv_pending = false;
     uint32_t kv_parity = 0;
+    // the low halves sit at columns j*d (Q) and H + j*d (K) of qk_lo
+    const int colQl = j * AHD, colKl = p.H + j * AHD;
     if (tid == 0) {
         tma_prefetch_desc(&tm);
-        mbar_arrive_expect_tx(bar_q, 2 * ATILE);
+        if (LO) tma_prefetch_desc(&tml);
+        mbar_arrive_expect_tx(bar_q, (LO ? 4 : 2) * ATILE);
         tma_load_2d(sQ, &tm, bar_q, colQ, start + q0);
         tma_load_2d(sQ + ATILE, &tm, bar_q, colQ + 64, start + q0);
-        mbar_arrive_expect_tx(bar_kv, 4 * ATILE);
+        if (LO) {
+            tma_load_2d(sQl, &tml, bar_q, colQl, start + q0);
+            tma_load_2d(sQl + ATILE, &tml, bar_q, colQl + 64, start + q0);
+        }
+        mbar_arrive_expect_tx(bar_kv, (LO ? 6 : 4) * ATILE);
         tma_load_2d(sK, &tm, bar_kv, colK, start);
         tma_load_2d(sK + ATILE, &tm, bar_kv, colK + 64, start);
         tma_load_2d(sV, &tm, bar_kv, colV, start);
         tma_load_2d(sV + ATILE, &tm, bar_kv, colV + 64, start);
+        if (LO) {
+            tma_load_2d(sKl, &tml, bar_kv, colKl, start);
+            tma_load_2d(sKl + ATILE, &tml, bar_kv, colKl + 64, start);
+        }
         q_pending = kv_pending = true;
     }
     constexpr uint32_t fmt = std::is_same<T, __half>::value ? 0u : 1u;
@@ -139,6 +157,12 @@ __global__ void __launch_bounds__(128) attn_tc_kernel(const __grid_constant__ CU
                 const uint64_t a = smem_desc_k128(smem_u32(sQ + (k >> 2) * ATILE)) + 2 * (k & 3);
                 const uint64_t bk = smem_desc_k128(smem_u32(sK + (k >> 2) * ATILE)) + 2 * (k & 3);
                 umma_f16(tmem, a, bk, idesc_s, k > 0 ? 1u : 0u);
+                if (LO) {
+                    const uint64_t al = smem_desc_k128(smem_u32(sQl + (k >> 2) * ATILE)) + 2 * (k & 3);
+                    const uint64_t bl = smem_desc_k128(smem_u32(sKl + (k >> 2) * ATILE)) + 2 * (k & 3);
+                    umma_f16(tmem, a, bl, idesc_s, 1u);
+                    umma_f16(tmem, al, bk, idesc_s, 1u);
+                }
             }
             umma_commit(bar_mma);
         }
@@ -216,11 +240,15 @@ __global__ void __launch_bounds__(128) attn_tc_kernel(const __grid_constant__ CU
         tc_fence_after();
         if (kb + 1 < n_kb && tid == 0) {
             const int y = start + (kb + 1) * ATK;
-            mbar_arrive_expect_tx(bar_kv, 4 * ATILE);
+            mbar_arrive_expect_tx(bar_kv, (LO ? 6 : 4) * ATILE);
             tma_load_2d(sK, &tm, bar_kv, colK, y);
             tma_load_2d(sK + ATILE, &tm, bar_kv, colK + 64, y);
             tma_load_2d(sV, &tm, bar_kv, colV, y);
             tma_load_2d(sV + ATILE, &tm, bar_kv, colV + 64, y);
+            if (LO) {
+                tma_load_2d(sKl, &tml, bar_kv, colKl, y);
+                tma_load_2d(sKl + ATILE, &tml, bar_kv, colKl + 64, y);
+            }
             kv_pending = true;
         }
     }
@@ -273,27 +301,47 @@ static PFN_cuTensorMapEncodeTiled_v12000 attn_encode_fn() {
     return fn;
 }
 
-bool attention_tc_supported(int dtype, int H, int n_heads, const void* qkv, const void* o, int qkv_rows) {
+bool attention_tc_supported(int dtype, int H, int n_heads, const void* qkv, const void* qk_lo, const void* o,
+                            int qkv_rows) {
     if (dtype != ENERGON_F16 && dtype != ENERGON_BF16) return false;
     if (n_heads <= 0 || H % n_heads != 0 || H / n_heads != AHD) return false;
-    if (((uintptr_t)qkv | (uintptr_t)o) % 16 != 0 || qkv_rows < 1) return false;
+    if (((uintptr_t)qkv | (uintptr_t)qk_lo | (uintptr_t)o) % 16 != 0 || qkv_rows < 1) return false;
     return attn_encode_fn() != nullptr;
 }
 
-cudaError_t launch_attention_tc(int dtype, const void* qkv, void* o, const int32_t* cu, int batch, int max_len, int H,
-                                int n_heads, int qkv_rows, int32_t* status, uint64_t timeout_ns, cudaStream_t st) {
-    if (batch <= 0 || max_len <= 0) return cudaSuccess;
-    CUtensorMap tm;
-    cuuint64_t dims[2] = {(cuuint64_t)3 * H, (cuuint64_t)qkv_rows};
-    cuuint64_t strides[1] = {(cuuint64_t)3 * H * 2};
+// [rows, cols] 16-bit tensor, box 64 x 128, 128-byte swizzle (the Q / K / V tiles).
+static CUresult attn_tmap(CUtensorMap* m, int dtype, const void* ptr, int64_t cols, int64_t rows) {
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
     cuuint32_t box[2] = {64, 128};
     cuuint32_t estr[2] = {1, 1};
     const CUtensorMapDataType dt =
         dtype == ENERGON_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-    CUresult rc = attn_encode_fn()(&tm, dt, 2, const_cast<void*>(qkv), dims, strides, box, estr,
-                                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (rc != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    return attn_encode_fn()(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+template <typename T, bool LO>
+static cudaError_t attn_tc_launch(const CUtensorMap& tm, const CUtensorMap& tml, const AttnTcParams& p, dim3 grid,
+                                  cudaStream_t st) {
+    cudaError_t e = prepare_smem((const void*)attn_tc_kernel<T, LO>, at_smem<LO>());
+    if (e != cudaSuccess) return e;
+    attn_tc_kernel<T, LO><<<grid, 128, at_smem<LO>(), st>>>(tm, tml, p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_attention_tc(int dtype, const void* qkv, const void* qk_lo, void* o, const int32_t* cu, int batch,
+                                int max_len, int H, int n_heads, int qkv_rows, int32_t* status, uint64_t timeout_ns,
+                                cudaStream_t st) {
+    if (batch <= 0 || max_len <= 0) return cudaSuccess;
+    CUtensorMap tm, tml;
+    if (attn_tmap(&tm, dtype, qkv, 3 * (int64_t)H, qkv_rows) != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    if (qk_lo != nullptr) {
+        if (attn_tmap(&tml, dtype, qk_lo, 2 * (int64_t)H, qkv_rows) != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    } else {
+        tml = tm;
+    }
     AttnTcParams p;
     p.cu = cu;
     p.out = o;
@@ -302,16 +350,11 @@ cudaError_t launch_attention_tc(int dtype, const void* qkv, void* o, const int32
     p.scale_log2e = (float)(1.4426950408889634 / sqrt((double)AHD));
     p.timeout_ns = timeout_ns;
     dim3 grid((max_len + ATQ - 1) / ATQ, n_heads, batch);
-    if (dtype == ENERGON_BF16) {
-        cudaError_t e = prepare_smem((const void*)attn_tc_kernel<__nv_bfloat16>, AT_SMEM);
-        if (e != cudaSuccess) return e;
-        attn_tc_kernel<__nv_bfloat16><<<grid, 128, AT_SMEM, st>>>(tm, p);
-    } else {
-        cudaError_t e = prepare_smem((const void*)attn_tc_kernel<__half>, AT_SMEM);
-        if (e != cudaSuccess) return e;
-        attn_tc_kernel<__half><<<grid, 128, AT_SMEM, st>>>(tm, p);
-    }
-    return cudaGetLastError();
+    if (dtype == ENERGON_BF16)
+        return qk_lo ? attn_tc_launch<__nv_bfloat16, true>(tm, tml, p, grid, st)
+                     : attn_tc_launch<__nv_bfloat16, false>(tm, tml, p, grid, st);
+    return qk_lo ? attn_tc_launch<__half, true>(tm, tml, p, grid, st)
+                 : attn_tc_launch<__half, false>(tm, tml, p, grid, st);
 }
 
 }  // namespace energon

@@ -88,9 +88,12 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 int64_t rows_alloc(int batch, int pad_len) { return (int64_t)align_up((size_t)batch * (size_t)pad_len, 256); }
 
 struct LayerWs {
-    void *a, *qkv, *o, *x1, *f;
-    float* p32;  // split-K partial sums (buffers of <= 128 rows only)
+    void *a, *qkv, *qk_lo, *o, *f;
+    float* x1;      // residual after attention, fp32
+    float* p32;     // split-K partial sums (buffers of <= 128 rows only)
     size_t p32_bytes;
+    float2* stats;  // folded LayerNorm: (rstd, mean * rstd) per row
+    float *fold_c, *fold_d;
     size_t bytes;
 };
 
@@ -109,17 +112,22 @@ LayerWs layer_ws_layout(const energon_layer_config& c, int batch, int pad_len, v
     size_t off = 0;
     LayerWs w;
     auto take = [&](size_t bytes) {
-        void* r = p ? p + off : nullptr;
+        void* r = (p && bytes) ? p + off : nullptr;
         off = align_up(off + bytes, 1024);
         return r;
     };
     w.a = take(R * H * e);
     w.qkv = take(R * 3 * H * e);
+    // low halves of Q | K: 16-bit types only (fp32 values need no second term)
+    w.qk_lo = take(c.dtype == ENERGON_F32 ? 0 : R * 2 * H * e);
     w.o = take(R * H * e);
-    w.x1 = take(R * H * e);
+    w.x1 = static_cast<float*>(take(R * H * sizeof(float)));
     w.f = take(R * F * e);
     w.p32_bytes = splitk_bytes(c, batch, pad_len);
     w.p32 = static_cast<float*>(take(w.p32_bytes));
+    w.stats = static_cast<float2*>(take(R * sizeof(float2)));
+    w.fold_c = static_cast<float*>(take(2 * 3 * H * sizeof(float)));
+    w.fold_d = w.fold_c ? w.fold_c + 3 * H : nullptr;
     w.bytes = off;
     return w;
 }
@@ -211,68 +219,75 @@ GemmArgs gemm_base(const energon_layer_config& c, const int32_t* cu, int batch, 
 }
 
 // Attention sub-layer on the rows described by cu (row starts; rows valid = cu[batch]):
-//   x1 = x + attention(LN1(x) W_qkv^T + b_qkv) W_o^T + b_o
-// With `padded` set, x is gathered from that [batch, max_len, H] tensor by the first
-// LayerNorm (transpose_padding_remove fused into it), which also writes the packed
-// rows to x (then the residual stream's buffer).
+//   x1 = x + attention(LN1(x) W_qkv^T + b_qkv) W_o^T + b_o      (x1 in fp32)
+// LN1 is folded into the QKV GEMM: the GEMM reads u = x * ln1_g and its epilogue applies
+// the row statistics and c = W_qkv ln1_g, d = b_qkv + W_qkv ln1_b; Q and K are kept as
+// two 16-bit terms (qkv holds the high, qk_lo the low halves) for the attention scores.
+// With `padded` set, x is gathered from that [batch, max_len, H] tensor by the folded
+// LayerNorm (transpose_padding_remove fused into it), which also writes the packed rows
+// to x (then the residual stream's buffer).
 int attention_sublayer(const energon_layer_config& c, const energon_layer_weights& w, const void* x,
-                       const int32_t* cu, int batch, int max_len, void* x1, int32_t* status, const LayerWs& ws,
+                       const int32_t* cu, int batch, int max_len, float* x1, int32_t* status, const LayerWs& ws,
                        cudaStream_t st, const void* padded = nullptr) {
     const int H = c.hidden;
     const int M_cap = batch * max_len;
     const int A_rows = (int)rows_alloc(batch, max_len);
     const int32_t* d_rows = cu + batch;
-    if (padded != nullptr) {
-        LnGather gth;
-        gth.cu = cu, gth.batch = batch, gth.pad_len = max_len, gth.copy = const_cast<void*>(x);
-        CK(traced("layernorm_remove", st,
-                  [&] {
-                      return launch_layernorm(c.dtype, padded, w.ln1_g, w.ln1_b, ws.a, d_rows, M_cap, H, c.ln_eps,
-                                              status, st, gth);
-                  }),
-           "ln1 + remove");
-    } else {
-        CK(traced("layernorm", st,
-                  [&] {
-                      return launch_layernorm(c.dtype, x, w.ln1_g, w.ln1_b, ws.a, d_rows, M_cap, H, c.ln_eps, status,
-                                              st);
-                  }),
-           "ln1");
-    }
+    LnGather gth;
+    if (padded != nullptr) gth.cu = cu, gth.batch = batch, gth.pad_len = max_len, gth.copy = const_cast<void*>(x);
+    CK(traced(padded ? "layernorm_remove" : "ln_fold", st,
+              [&] {
+                  return launch_ln_fold(c.dtype, padded ? padded : x, w.ln1_g, ws.a, ws.stats, d_rows, M_cap, H,
+                                        c.ln_eps, status, st, gth);
+              }),
+       padded ? "ln1 fold + remove" : "ln1 fold");
+    CK(traced("ln_fold_weights", st,
+              [&] {
+                  return launch_ln_fold_weights(c.dtype, w.w_qkv, w.ln1_g, w.ln1_b, w.b_qkv, 3 * H, H, ws.fold_c,
+                                                ws.fold_d, status, st);
+              }),
+       "ln1 fold weights");
     GemmArgs g = gemm_base(c, cu, batch, max_len, status, ws);
-    g.A = ws.a, g.W = w.w_qkv, g.bias = w.b_qkv, g.residual = nullptr, g.out = ws.qkv;
-    g.N = 3 * H, g.K = H, g.epilogue = EPI_BIAS;
+    g.A = ws.a, g.W = w.w_qkv, g.bias = nullptr, g.residual = nullptr, g.out = ws.qkv;
+    g.N = 3 * H, g.K = H, g.epilogue = EPI_LN_FOLD;
+    g.fold_stats = ws.stats, g.fold_c = ws.fold_c, g.fold_d = ws.fold_d;
+    g.lo = ws.qk_lo, g.lo_cols = ws.qk_lo ? 2 * H : 0;
     if (int r = run_gemm(g, st, "gemm_qkv")) return r;
     CK(traced("attention", st,
               [&] {
-                  return launch_attention(c.dtype, ws.qkv, ws.o, cu, batch, max_len, H, c.n_heads, A_rows, status,
-                                          g_timeout_ns, st);
+                  return launch_attention(c.dtype, ws.qkv, ws.qk_lo, ws.o, cu, batch, max_len, H, c.n_heads, A_rows,
+                                          status, g_timeout_ns, st);
               }),
        "attention");
+    g = gemm_base(c, cu, batch, max_len, status, ws);
     g.A = ws.o, g.W = w.w_o, g.bias = w.b_o, g.residual = x, g.out = x1;
-    g.N = H, g.K = H, g.epilogue = EPI_BIAS_RESIDUAL;
+    g.N = H, g.K = H, g.epilogue = EPI_RES_OUT32;
     return run_gemm(g, st, "gemm_out_proj");
 }
 
-// MLP sub-layer: y = x1 + GELU(LN2(x1) W_1^T + b_1) W_2^T + b_2 (y may alias nothing but itself).
-// With `padded_out` set and the FFN2 GEMM on the CTA-pair kernel, its epilogue stores each
-// row at its padded position in padded_out (transpose_padding_rebuild fused into it; pad
-// rows are left alone) and *scattered is set; otherwise the rows go to y.
-int mlp_sublayer(const energon_layer_config& c, const energon_layer_weights& w, const void* x1, const int32_t* cu,
+// MLP sub-layer: y = x1 + GELU(LN2(x1) W_1^T + b_1) W_2^T + b_2, x1 in fp32, y in the
+// storage type (y may alias nothing but itself).  With `padded_out` set and the FFN2 GEMM
+// on the CTA-pair kernel, its epilogue stores each row at its padded position in
+// padded_out (transpose_padding_rebuild fused into it; pad rows are left alone) and
+// *scattered is set; otherwise the rows go to y.
+int mlp_sublayer(const energon_layer_config& c, const energon_layer_weights& w, const float* x1, const int32_t* cu,
                  int batch, int max_len, void* y, int32_t* status, const LayerWs& ws, cudaStream_t st,
                  void* padded_out = nullptr, bool* scattered = nullptr) {
     const int H = c.hidden, F = c.ffn;
     const int M_cap = batch * max_len;
     const int32_t* d_rows = cu + batch;
     CK(traced("layernorm", st,
-              [&] { return launch_layernorm(c.dtype, x1, w.ln2_g, w.ln2_b, ws.a, d_rows, M_cap, H, c.ln_eps, status, st); }),
+              [&] {
+                  return launch_layernorm(c.dtype, x1, w.ln2_g, w.ln2_b, ws.a, d_rows, M_cap, H, c.ln_eps, status, st,
+                                          LnGather(), true);
+              }),
        "ln2");
     GemmArgs g = gemm_base(c, cu, batch, max_len, status, ws);
     g.A = ws.a, g.W = w.w_1, g.bias = w.b_1, g.residual = nullptr, g.out = ws.f;
     g.N = F, g.K = H, g.epilogue = EPI_BIAS_GELU;
     if (int r = run_gemm(g, st, "gemm_ffn1")) return r;
     g.A = ws.f, g.W = w.w_2, g.bias = w.b_2, g.residual = x1, g.out = y;
-    g.N = H, g.K = F, g.epilogue = EPI_BIAS_RESIDUAL;
+    g.N = H, g.K = F, g.epilogue = EPI_RES32;
     if (scattered) *scattered = false;
     if (padded_out != nullptr) {
         GemmArgs gs = g;
@@ -468,15 +483,17 @@ int energon_stack_forward(const energon_layer_config* cfg, const energon_layer_w
         CK(traced("padded_starts", st, [&] { return launch_padded_starts(batch, pad_len, ws.cu_pad, d_status, st); }),
            "padded starts");
         const void* src = padded_in;
-        void* x1_pk = ws.layer.o;    // free once the out-projection has consumed it
-        void* y_pk = ws.layer.qkv;   // free once attention has consumed it
+        float* x1_pk = static_cast<float*>(ws.layer.qkv);   // free once attention has consumed it
+        void* y_pk = ws.layer.o;                            // free once the out-projection has consumed it
+        const int64_t x1_row_bytes = (int64_t)cfg->hidden * (int64_t)sizeof(float);
         for (int l = 0; l < n_layers; ++l) {
             if (int r = attention_sublayer(*cfg, layers[l], src, ws.cu_pad, batch, pad_len, ws.layer.x1, d_status,
                                            ws.layer, st))
                 return r;
             CK(traced("remove_padding", st,
                       [&] {
-                          return launch_remove(ws.layer.x1, ws.cu, batch, pad_len, row_bytes, x1_pk, R, d_status, st);
+                          return launch_remove(ws.layer.x1, ws.cu, batch, pad_len, x1_row_bytes, x1_pk, R, d_status,
+                                               st);
                       }),
                "remove");
             if (int r = mlp_sublayer(*cfg, layers[l], x1_pk, ws.cu, batch, pad_len, y_pk, d_status, ws.layer, st))

@@ -1,9 +1,10 @@
-// CUDA-core GEMM y = A W^T + bias (+ GELU) (+ residual) for the fp32 layer and
-// for shapes the tcgen05 kernel does not take.  64 x 64 output tile per
-// 256-thread block, 4 x 4 outputs per thread, K staged through shared memory
-// in steps of 16.  Same epilogue semantics as the tensor-core kernel: fp32
-// accumulate, bias, optional GELU, optional residual, one rounding to the
-// storage type.  The valid row count is read on the device.
+// CUDA-core GEMM y = A W^T + epilogue for the fp32 layer and for shapes the
+// tcgen05 kernel does not take.  64 x 64 output tile per 256-thread block,
+// 4 x 4 outputs per thread, K staged through shared memory in steps of 16.
+// Same epilogue semantics as the tensor-core kernel (the Epilogue enum): fp32
+// accumulate, then the folded LayerNorm or bias, optional GELU, optional
+// residual, one rounding to the output type.  The valid row count is read on
+// the device.
 #include "common.cuh"
 #include "internal.h"
 
@@ -15,13 +16,12 @@ constexpr int SBM = 64, SBN = 64, SBK = 16;
 
 template <typename T, int EPI>
 __global__ void __launch_bounds__(256) gemm_simt_kernel(const T* __restrict__ A, const T* __restrict__ W,
-                                                        const T* __restrict__ bias, const T* residual, T* out,
-                                                        const int32_t* d_rows, int M_cap, int N, int K, int gelu_tanh,
-                                                        const int32_t* status) {
+                                                        const GemmArgs a) {
     __shared__ float As[SBK][SBM + 4];
     __shared__ float Ws[SBK][SBN + 4];
-    if (status_bad(status)) return;
-    const int M = min(*d_rows, M_cap);
+    if (status_bad(a.status)) return;
+    const int M = min(*a.d_rows, a.M_cap);
+    const int N = a.N, K = a.K;
     const int m0 = blockIdx.y * SBM, n0 = blockIdx.x * SBN;
     if (m0 >= M) return;
     const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
@@ -40,32 +40,44 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(const T* __restrict__ A,
         __syncthreads();
 #pragma unroll
         for (int k = 0; k < SBK; ++k) {
-            float a[4], b[4];
+            float av[4], bv[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                a[i] = As[k][ty * 4 + i];
-                b[i] = Ws[k][tx * 4 + i];
+                av[i] = As[k][ty * 4 + i];
+                bv[i] = Ws[k][tx * 4 + i];
             }
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
         }
         __syncthreads();
     }
+    const T* bias = static_cast<const T*>(a.bias);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int gm = m0 + ty * 4 + i;
         if (gm >= M) continue;
+        const float2 fs = EPI == EPI_LN_FOLD ? a.fold_stats[gm] : make_float2(0.0f, 0.0f);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int gn = n0 + tx * 4 + j;
             if (gn >= N) continue;
+            const int64_t o = (int64_t)gm * N + gn;
             float v = acc[i][j];
-            if (bias) v += to_f(bias[gn]);
-            if (EPI == EPI_BIAS_GELU) v = gelu_f(v, gelu_tanh != 0);
-            if (EPI == EPI_BIAS_RESIDUAL) v += to_f(residual[(int64_t)gm * N + gn]);
-            out[(int64_t)gm * N + gn] = from_f<T>(v);
+            if (EPI == EPI_LN_FOLD) v = fmaf(v, fs.x, fmaf(-fs.y, a.fold_c[gn], a.fold_d[gn]));
+            else if (bias) v += to_f(bias[gn]);
+            if (EPI == EPI_BIAS_GELU) v = gelu_f(v, a.gelu_tanh != 0);
+            if (EPI == EPI_BIAS_RESIDUAL || EPI == EPI_RES_OUT32) v += to_f(static_cast<const T*>(a.residual)[o]);
+            if (EPI == EPI_RES32) v += static_cast<const float*>(a.residual)[o];
+            if (EPI == EPI_RES_OUT32) {
+                static_cast<float*>(a.out)[o] = v;
+            } else {
+                const T h = from_f<T>(v);
+                static_cast<T*>(a.out)[o] = h;
+                if (EPI == EPI_LN_FOLD && a.lo != nullptr && gn < a.lo_cols)
+                    static_cast<T*>(a.lo)[(int64_t)gm * a.lo_cols + gn] = from_f<T>(v - to_f(h));
+            }
         }
     }
 }
@@ -73,21 +85,14 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(const T* __restrict__ A,
 template <typename T>
 static void simt_dispatch(const GemmArgs& a, cudaStream_t st) {
     dim3 grid((a.N + SBN - 1) / SBN, (a.M_cap + SBM - 1) / SBM);
-    const T *A = (const T*)a.A, *W = (const T*)a.W, *b = (const T*)a.bias, *r = (const T*)a.residual;
-    T* o = (T*)a.out;
+    const T *A = (const T*)a.A, *W = (const T*)a.W;
     switch (a.epilogue) {
-    case EPI_BIAS:
-        gemm_simt_kernel<T, EPI_BIAS><<<grid, 256, 0, st>>>(A, W, b, r, o, a.d_rows, a.M_cap, a.N, a.K, a.gelu_tanh,
-                                                            a.status);
-        break;
-    case EPI_BIAS_GELU:
-        gemm_simt_kernel<T, EPI_BIAS_GELU><<<grid, 256, 0, st>>>(A, W, b, r, o, a.d_rows, a.M_cap, a.N, a.K,
-                                                                 a.gelu_tanh, a.status);
-        break;
-    default:
-        gemm_simt_kernel<T, EPI_BIAS_RESIDUAL><<<grid, 256, 0, st>>>(A, W, b, r, o, a.d_rows, a.M_cap, a.N, a.K,
-                                                                     a.gelu_tanh, a.status);
-        break;
+    case EPI_BIAS: gemm_simt_kernel<T, EPI_BIAS><<<grid, 256, 0, st>>>(A, W, a); break;
+    case EPI_BIAS_GELU: gemm_simt_kernel<T, EPI_BIAS_GELU><<<grid, 256, 0, st>>>(A, W, a); break;
+    case EPI_BIAS_RESIDUAL: gemm_simt_kernel<T, EPI_BIAS_RESIDUAL><<<grid, 256, 0, st>>>(A, W, a); break;
+    case EPI_LN_FOLD: gemm_simt_kernel<T, EPI_LN_FOLD><<<grid, 256, 0, st>>>(A, W, a); break;
+    case EPI_RES_OUT32: gemm_simt_kernel<T, EPI_RES_OUT32><<<grid, 256, 0, st>>>(A, W, a); break;
+    default: gemm_simt_kernel<T, EPI_RES32><<<grid, 256, 0, st>>>(A, W, a); break;
     }
 }
 

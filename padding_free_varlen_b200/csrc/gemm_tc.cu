@@ -65,6 +65,12 @@ struct TcParams {
     // goes to padded row b * scatter_pad_len + r - scatter_cu[b] of a [batch, pad_len, N] tensor
     const int32_t* scatter_cu;
     int scatter_batch, scatter_pad_len;
+    // EPI_LN_FOLD: per-row (rstd, mean * rstd), per-column c and d, low halves [M_cap, lo_cols]
+    const float2* fold_stats;
+    const float* fold_c;
+    const float* fold_d;
+    void* lo;
+    int lo_cols;
 };
 
 // Destination row of packed row `row` (its padded position when the epilogue scatters).
@@ -114,15 +120,57 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
     return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
-// Bias, optional GELU, optional residual (already loaded by the caller into `res`),
-// one rounding to T, 64-byte store of 32 consecutive columns of one row.
+// ------------------------------------------------------------------ epilogue
+//
+// Per 32-column chunk of one output row (the accumulator columns a thread holds):
+//   EPI_LN_FOLD    v = rstd acc - (mean rstd) c + d; columns below lo_cols also store
+//                  the low half round(v - round(v)) to `lo`
+//   EPI_BIAS_GELU  v = GELU(acc + bias)
+//   EPI_RES_OUT32  v = acc + bias + residual (storage type), stored as fp32
+//   EPI_RES32      v = acc + bias + residual (fp32), stored in the storage type
+// One rounding to the output type at the end.
+
+template <int EPI>
+struct Epi {
+    static constexpr bool FOLD = EPI == EPI_LN_FOLD;
+    static constexpr bool GELU = EPI == EPI_BIAS_GELU;
+    static constexpr bool RES_T = EPI == EPI_RES_OUT32;   // residual in the storage type
+    static constexpr bool RES_F32 = EPI == EPI_RES32;     // residual in fp32
+    static constexpr bool OUT_F32 = EPI == EPI_RES_OUT32;
+    static constexpr int RES_VECS = RES_F32 ? 8 : (RES_T ? 4 : 0);  // 16-byte vectors per 32 columns
+};
+
+// Residual of one row's 32 columns [col0, col0 + 32), read straight from global memory.
 template <typename T, int EPI>
-__device__ __forceinline__ void epilogue_store32(const uint32_t* acc, const uint4* res, const TcParams& p,
-                                                 int64_t out_row, int col0) {
-    float v[32];
+__device__ __forceinline__ void load_residual32(const TcParams& p, int row, int col0, bool live, uint4* res) {
+    constexpr int NV = Epi<EPI>::RES_VECS;
+    if (NV > 0 && live) {
+        const size_t eb = Epi<EPI>::RES_F32 ? 4 : sizeof(T);
+        const uint4* rp = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.residual) +
+                                                         ((size_t)row * p.N + col0) * eb);
+#pragma unroll
+        for (int q = 0; q < NV; ++q) res[q] = rp[q];
+    }
+}
+
+// Accumulator chunk -> final fp32 values (before the one rounding).
+template <typename T, int EPI>
+__device__ __forceinline__ void epi_math(float* v, const uint32_t* acc, const TcParams& p, int col0, float2 fs,
+                                         const uint4* res) {
 #pragma unroll
     for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(acc[j]);
-    if (p.bias != nullptr) {
+    if (Epi<EPI>::FOLD) {
+        const float4* cp = reinterpret_cast<const float4*>(p.fold_c + col0);
+        const float4* dp = reinterpret_cast<const float4*>(p.fold_d + col0);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const float4 c = __ldg(cp + q), d = __ldg(dp + q);
+            v[4 * q + 0] = fmaf(v[4 * q + 0], fs.x, fmaf(-fs.y, c.x, d.x));
+            v[4 * q + 1] = fmaf(v[4 * q + 1], fs.x, fmaf(-fs.y, c.y, d.y));
+            v[4 * q + 2] = fmaf(v[4 * q + 2], fs.x, fmaf(-fs.y, c.z, d.z));
+            v[4 * q + 3] = fmaf(v[4 * q + 3], fs.x, fmaf(-fs.y, c.w, d.w));
+        }
+    } else if (p.bias != nullptr) {
         const uint4* bp = reinterpret_cast<const uint4*>(static_cast<const T*>(p.bias) + col0);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -136,7 +184,7 @@ __device__ __forceinline__ void epilogue_store32(const uint32_t* acc, const uint
             }
         }
     }
-    if (EPI == EPI_BIAS_GELU) {
+    if (Epi<EPI>::GELU) {
         if (p.gelu_tanh) {
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = gelu_tanh_fast(v[j]);
@@ -145,7 +193,7 @@ __device__ __forceinline__ void epilogue_store32(const uint32_t* acc, const uint
             for (int j = 0; j < 32; ++j) v[j] = gelu_f(v[j], false);
         }
     }
-    if (EPI == EPI_BIAS_RESIDUAL) {
+    if (Epi<EPI>::RES_T) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
             const uint32_t* ww = reinterpret_cast<const uint32_t*>(&res[q]);
@@ -157,139 +205,179 @@ __device__ __forceinline__ void epilogue_store32(const uint32_t* acc, const uint
             }
         }
     }
-    uint4* op = reinterpret_cast<uint4*>(static_cast<T*>(p.out) + out_row * p.N + col0);
+    if (Epi<EPI>::RES_F32) {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        uint4 o;
-        o.x = pack2<T>(v[q * 8 + 0], v[q * 8 + 1]);
-        o.y = pack2<T>(v[q * 8 + 2], v[q * 8 + 3]);
-        o.z = pack2<T>(v[q * 8 + 4], v[q * 8 + 5]);
-        o.w = pack2<T>(v[q * 8 + 6], v[q * 8 + 7]);
-        op[q] = o;
+        for (int q = 0; q < 8; ++q) {
+            v[4 * q + 0] += __uint_as_float(res[q].x);
+            v[4 * q + 1] += __uint_as_float(res[q].y);
+            v[4 * q + 2] += __uint_as_float(res[q].z);
+            v[4 * q + 3] += __uint_as_float(res[q].w);
+        }
     }
 }
 
+// 32 values -> 4 words of two storage-type elements each (hi), and the low halves.
+template <typename T>
+__device__ __forceinline__ uint4 pack8(const float* v) {
+    uint4 o;
+    o.x = pack2<T>(v[0], v[1]);
+    o.y = pack2<T>(v[2], v[3]);
+    o.z = pack2<T>(v[4], v[5]);
+    o.w = pack2<T>(v[6], v[7]);
+    return o;
+}
+// The low half of a two-term value: round(v - round(v)); v - round(v) is exact in fp32.
+template <typename T>
+__device__ __forceinline__ uint32_t pack2_lo(float a, float b, uint32_t hi) {
+    const float2 h = unpack2<T>(hi);
+    return pack2<T>(a - h.x, b - h.y);
+}
+template <typename T>
+__device__ __forceinline__ uint4 pack8_lo(const float* v, uint4 hi) {
+    uint4 o;
+    o.x = pack2_lo<T>(v[0], v[1], hi.x);
+    o.y = pack2_lo<T>(v[2], v[3], hi.y);
+    o.z = pack2_lo<T>(v[4], v[5], hi.z);
+    o.w = pack2_lo<T>(v[6], v[7], hi.w);
+    return o;
+}
+
+// Row-per-thread store of one chunk (the path for rows past a full 32-row box).
 template <typename T, int EPI>
-__device__ __forceinline__ void load_residual32(const TcParams& p, int row, int col0, bool live, uint4* res) {
-    if (EPI == EPI_BIAS_RESIDUAL && live) {
-        const uint4* rp = reinterpret_cast<const uint4*>(static_cast<const T*>(p.residual) + (int64_t)row * p.N + col0);
+__device__ __forceinline__ void epilogue_store32(uint32_t* acc, const uint4* res, const TcParams& p, int row,
+                                                 int64_t out_row, int col0, float2 fs) {
+    float* v = reinterpret_cast<float*>(acc);  // the values replace the accumulator bits
+    epi_math<T, EPI>(v, acc, p, col0, fs, res);
+    if (Epi<EPI>::OUT_F32) {
+        float4* op = reinterpret_cast<float4*>(static_cast<float*>(p.out) + out_row * p.N + col0);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) res[q] = rp[q];
+        for (int q = 0; q < 8; ++q) op[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        return;
+    }
+    uint4* op = reinterpret_cast<uint4*>(static_cast<T*>(p.out) + out_row * p.N + col0);
+    const bool lo = Epi<EPI>::FOLD && p.lo != nullptr && col0 < p.lo_cols;
+    uint4* lp = lo ? reinterpret_cast<uint4*>(static_cast<T*>(p.lo) + (int64_t)row * p.lo_cols + col0) : nullptr;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const uint4 h = pack8<T>(v + 8 * q);
+        op[q] = h;
+        if (lo) lp[q] = pack8_lo<T>(v + 8 * q, h);
     }
 }
 
 // One warp drains 256 accumulator columns of its 32 TMEM lanes (= 32 output rows),
-// 32 columns at a time; the TMEM load and the residual load of the next chunk are
-// issued before the current chunk is processed.
+// 32 columns at a time, row per thread; the TMEM load and the residual load of the next
+// chunk are issued before the current chunk is processed.
 template <typename T, int EPI>
 __device__ __forceinline__ void drain_256(uint32_t tbase, const TcParams& p, int row, int col_base, int M) {
+    // The path for the one box per tile that holds row M - 1 (and boxes that straddle two
+    // sequences when scattering): the residual is loaded chunk by chunk, not ahead.
+    constexpr int NV = Epi<EPI>::RES_VECS > 0 ? Epi<EPI>::RES_VECS : 1;
     uint32_t r[2][32];
-    uint4 res[2][4];
+    uint4 res[NV];
     const bool row_ok = row < M;
     const int64_t out_row = row_ok ? out_row_of(p, row) : 0;
+    const float2 fs = (Epi<EPI>::FOLD && row_ok) ? p.fold_stats[row] : make_float2(0.0f, 0.0f);
     tmem_ld_x16(tbase, r[0]);
     tmem_ld_x16(tbase + 16, r[0] + 16);
-    load_residual32<T, EPI>(p, row, col_base, row_ok && col_base < p.N, res[0]);
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
         const int cur = c & 1;
+        const int col0 = col_base + c * 32;
+        const bool live = row_ok && col0 < p.N;
+        load_residual32<T, EPI>(p, row, col0, live, res);
         tmem_wait_ld_regs(r[cur]);
         if (c + 1 < 8) {
             tmem_ld_x16(tbase + (c + 1) * 32, r[cur ^ 1]);
             tmem_ld_x16(tbase + (c + 1) * 32 + 16, r[cur ^ 1] + 16);
-            const int coln = col_base + (c + 1) * 32;
-            load_residual32<T, EPI>(p, row, coln, row_ok && coln < p.N, res[cur ^ 1]);
         }
-        const int col0 = col_base + c * 32;
-        if (row_ok && col0 < p.N) epilogue_store32<T, EPI>(r[cur], res[cur], p, out_row, col0);
+        if (live) epilogue_store32<T, EPI>(r[cur], res, p, row, out_row, col0, fs);
     }
 }
 
-// Staging buffer of one epilogue warp: 32 rows x 32 columns of 16-bit values,
-// 64 bytes per row, in the TMA 64-byte swizzle (the 16-byte chunk index is XORed
-// with bits 1-2 of the row), so that 32 threads each touching their own row hit
-// every bank once per 128 bytes.
+// Staging buffer of one epilogue warp: 32 rows x 64 bytes (32 columns of 16-bit values,
+// or 16 of fp32), in the TMA 64-byte swizzle (the 16-byte chunk index is XORed with bits
+// 1-2 of the row), so that 32 threads each touching their own row hit every bank once
+// per 128 bytes.
 __device__ __forceinline__ uint32_t stage_off(int row, int chunk) {
     return (uint32_t)(row * 64 + ((chunk ^ ((row >> 1) & 3)) << 4));
 }
 
-// One warp drains 256 accumulator columns of its 32 rows through shared memory:
-// per 32-column chunk, TMEM -> registers -> bias / GELU / residual -> one
-// rounding -> the warp's staging buffer -> one TMA store of the 32 x 32 box.
-// The residual box of the next chunk is fetched by TMA into the other buffer
-// while the current one is processed.  The accumulator is handed back (arrival
-// on `tempty_cluster`) as soon as its last columns are in registers.  Every row
-// of the warp must be valid (rows < M); the warp holding the last valid row
-// takes drain_256 instead.  Returns false if a residual copy timed out.
+// One warp drains 256 accumulator columns of its 32 rows through shared memory: per
+// 32-column chunk, TMEM -> registers -> epilogue math -> one rounding -> a staging
+// buffer -> one TMA store of the 32 x 32 box (and, for the low halves, a second box
+// from the other buffer).  Residuals in the storage type are fetched by TMA into the
+// other buffer one chunk ahead; fp32 residuals are loaded into registers one chunk
+// ahead; fp32 outputs are stored straight from registers, each thread writing whole
+// 128-byte lines of its row.  The accumulator is handed back (arrival on
+// `tempty_cluster`) as soon as its last columns are in registers.  Every row of the
+// warp must be valid (rows < M); the warp holding the last valid row takes drain_256
+// instead.  Returns false if a residual copy timed out.
 template <typename T, int EPI>
 __device__ __forceinline__ bool drain_256_staged(uint32_t tbase, const TcParams& p, const CUtensorMap* tmO,
-                                                 const CUtensorMap* tmR, uint8_t* sbuf, uint64_t* rbar,
-                                                 uint32_t& rpar, int row_base, int out_row_base, int col_base,
-                                                 uint32_t tempty_cluster, const volatile int* abort_flag) {
+                                                 const CUtensorMap* tmR, const CUtensorMap* tmL, uint8_t* sbuf,
+                                                 uint64_t* rbar, uint32_t& rpar, int row_base, int out_row_base,
+                                                 int col_base, uint32_t tempty_cluster,
+                                                 const volatile int* abort_flag) {
+    using E = Epi<EPI>;
+    constexpr bool TMA_RES = E::RES_T;                 // residual boxes through shared memory
+    constexpr int NV = E::RES_F32 ? 8 : 1;
+    // With fp32 residuals in registers (two chunks' worth), the accumulator chunk is not
+    // double-buffered: each chunk's TMEM load is issued and awaited in its own iteration.
+    constexpr int RB = E::RES_F32 ? 1 : 2;
     const int lane = threadIdx.x & 31;
-    uint32_t r[2][32];
+    const int row = row_base + lane;
+    const bool lo = E::FOLD && p.lo != nullptr && col_base < p.lo_cols;   // uniform over the tile
+    uint32_t r[RB][32];
+    uint4 res[2][NV];
     bool ok = true;
     uint32_t pend = 0;  // buffers with a residual copy in flight
+    const float2 fs = E::FOLD ? p.fold_stats[row] : make_float2(0.0f, 0.0f);
     if (lane == 0) {
         bulk_wait_read<0>();  // the previous tile's stores no longer read either buffer
-        if (EPI == EPI_BIAS_RESIDUAL) {
+        if (TMA_RES) {
             mbar_arrive_expect_tx(&rbar[0], 32 * 64);
             tma_load_2d(sbuf, tmR, &rbar[0], col_base, row_base);
         }
     }
-    if (EPI == EPI_BIAS_RESIDUAL) pend = 1u;
+    if (TMA_RES) pend = 1u;
     __syncwarp();
-    tmem_ld_x16(tbase, r[0]);
-    tmem_ld_x16(tbase + 16, r[0] + 16);
+    if (E::RES_F32) load_residual32<T, EPI>(p, row, col_base, true, res[0]);
+    if (RB == 2) {
+        tmem_ld_x16(tbase, r[0]);
+        tmem_ld_x16(tbase + 16, r[0] + 16);
+    }
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
         const int cur = c & 1;
+        const int rc = RB == 2 ? cur : 0;
         uint8_t* buf = sbuf + cur * 2048;
-        tmem_wait_ld_regs(r[cur]);
+        if (RB == 1) {
+            tmem_ld_x16(tbase + c * 32, r[0]);
+            tmem_ld_x16(tbase + c * 32 + 16, r[0] + 16);
+            if (c + 1 < 8) load_residual32<T, EPI>(p, row, col_base + (c + 1) * 32, true, res[cur ^ 1]);
+        }
+        tmem_wait_ld_regs(r[rc]);
         if (c + 1 < 8) {
-            tmem_ld_x16(tbase + (c + 1) * 32, r[cur ^ 1]);
-            tmem_ld_x16(tbase + (c + 1) * 32 + 16, r[cur ^ 1] + 16);
+            if (RB == 2) {
+                tmem_ld_x16(tbase + (c + 1) * 32, r[rc ^ 1]);
+                tmem_ld_x16(tbase + (c + 1) * 32 + 16, r[rc ^ 1] + 16);
+            }
         } else {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(tempty_cluster);
         }
         const int col0 = col_base + c * 32;
-        if (EPI == EPI_BIAS_RESIDUAL && c + 1 < 8) {
+        if (TMA_RES && c + 1 < 8) {
             if (lane == 0) {
-                bulk_wait_read<0>();  // chunk c-1's store has read the other buffer
                 mbar_arrive_expect_tx(&rbar[cur ^ 1], 32 * 64);
                 tma_load_2d(sbuf + (cur ^ 1) * 2048, tmR, &rbar[cur ^ 1], col0 + 32, row_base);
             }
             pend |= 1u << (cur ^ 1);
         }
-        float v[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[cur][j]);
-        if (p.bias != nullptr) {
-            const uint4* bp = reinterpret_cast<const uint4*>(static_cast<const T*>(p.bias) + col0);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const uint4 w = __ldg(bp + q);
-                const uint32_t* ww = reinterpret_cast<const uint32_t*>(&w);
-#pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    const float2 f = unpack2<T>(ww[h]);
-                    v[q * 8 + 2 * h] += f.x;
-                    v[q * 8 + 2 * h + 1] += f.y;
-                }
-            }
-        }
-        if (EPI == EPI_BIAS_GELU) {
-            if (p.gelu_tanh) {
-#pragma unroll
-                for (int j = 0; j < 32; ++j) v[j] = gelu_tanh_fast(v[j]);
-            } else {
-#pragma unroll
-                for (int j = 0; j < 32; ++j) v[j] = gelu_f(v[j], false);
-            }
-        }
-        if (EPI == EPI_BIAS_RESIDUAL) {
+        uint4 rt[4];
+        if (TMA_RES) {
             const bool got = mbar_wait_bounded(&rbar[cur], (rpar >> cur) & 1u, abort_flag, p.timeout_ns);
             if (!__all_sync(0xffffffffu, got)) {
                 // copies still in flight get one more bounded wait before the warp gives up
@@ -302,29 +390,47 @@ __device__ __forceinline__ bool drain_256_staged(uint32_t tbase, const TcParams&
             rpar ^= 1u << cur;
             pend &= ~(1u << cur);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const uint4 w = *reinterpret_cast<const uint4*>(buf + stage_off(lane, q));
-                const uint32_t* ww = reinterpret_cast<const uint32_t*>(&w);
+            for (int q = 0; q < 4; ++q) rt[q] = *reinterpret_cast<const uint4*>(buf + stage_off(lane, q));
+            // every lane has read this buffer before lane 0 refills it (two chunks on)
+            fence_proxy_async_smem();
+            __syncwarp();
+        }
+        float* v = reinterpret_cast<float*>(r[rc]);  // the chunk's values replace its accumulator bits
+        epi_math<T, EPI>(v, r[rc], p, col0, fs, TMA_RES ? rt : res[cur]);
+        if (E::OUT_F32) {
+            float4* op = reinterpret_cast<float4*>(static_cast<float*>(p.out) + (int64_t)(out_row_base + lane) * p.N + col0);
 #pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    const float2 f = unpack2<T>(ww[h]);
-                    v[q * 8 + 2 * h] += f.x;
-                    v[q * 8 + 2 * h + 1] += f.y;
-                }
+            for (int q = 0; q < 8; ++q) op[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+            continue;
+        }
+        if (lo) {
+            // both buffers take this chunk (high and low halves): the previous chunk's two
+            // stores must have read them
+            if (lane == 0) bulk_wait_read<0>();
+            __syncwarp();
+            uint8_t* b0 = sbuf;
+            uint8_t* b1 = sbuf + 2048;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const uint4 h = pack8<T>(v + 8 * q);
+                *reinterpret_cast<uint4*>(b0 + stage_off(lane, q)) = h;
+                *reinterpret_cast<uint4*>(b1 + stage_off(lane, q)) = pack8_lo<T>(v + 8 * q, h);
             }
-        } else if (c >= 2) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_2d(tmO, b0, col0, out_row_base);
+                tma_store_2d(tmL, b1, col0, row_base);
+                bulk_commit();
+            }
+            continue;
+        }
+        if (c >= 2) {
             if (lane == 0) bulk_wait_read<1>();  // chunk c-2's store has read this buffer
             __syncwarp();
         }
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            uint4 o;
-            o.x = pack2<T>(v[q * 8 + 0], v[q * 8 + 1]);
-            o.y = pack2<T>(v[q * 8 + 2], v[q * 8 + 3]);
-            o.z = pack2<T>(v[q * 8 + 4], v[q * 8 + 5]);
-            o.w = pack2<T>(v[q * 8 + 6], v[q * 8 + 7]);
-            *reinterpret_cast<uint4*>(buf + stage_off(lane, q)) = o;
-        }
+        for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(buf + stage_off(lane, q)) = pack8<T>(v + 8 * q);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
@@ -352,59 +458,41 @@ __device__ __forceinline__ void drain_256_partial(uint32_t tbase, float* part, i
     }
 }
 
-// Split-K finish: out[row][col] = epilogue(sum over s = 0 .. S-1 of partials[s][row][col]),
-// the splits summed in index order (deterministic), 8 columns per thread.
+// Split-K finish: out[row][cols] = epilogue(sum over s = 0 .. S-1 of partials[s][row][cols]),
+// the splits summed in index order (deterministic), 32 columns per thread, through the
+// same epilogue code as the tile kernels.
 template <typename T, int EPI>
-__global__ void __launch_bounds__(256) splitk_finish_kernel(const float* __restrict__ partials, int S, int M_cap,
-                                                            const int32_t* d_rows, int N, const T* __restrict__ bias,
-                                                            const T* residual, T* out, int gelu_tanh,
-                                                            const int32_t* status) {
-    if (status_bad(status)) return;
-    const int M = min(*d_rows, M_cap);
-    const int vec_per_row = N / 8;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)M * vec_per_row;
+__global__ void __launch_bounds__(256) splitk_finish_kernel(const float* __restrict__ partials, int S, TcParams p) {
+    if (status_bad(p.status)) return;
+    const int M = min(*p.d_rows, p.M_cap);
+    const int chunks = p.N / 32;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)M * chunks;
          i += (int64_t)gridDim.x * blockDim.x) {
-        const int row = (int)(i / vec_per_row), col0 = (int)(i % vec_per_row) * 8;
-        float v[8];
-        const float4* p0 = reinterpret_cast<const float4*>(partials + (int64_t)row * N + col0);
-        float4 a = p0[0], b = p0[1];
-        v[0] = a.x, v[1] = a.y, v[2] = a.z, v[3] = a.w, v[4] = b.x, v[5] = b.y, v[6] = b.z, v[7] = b.w;
+        const int row = (int)(i / chunks), col0 = (int)(i % chunks) * 32;
+        uint32_t acc[32];
+        const float4* p0 = reinterpret_cast<const float4*>(partials + (int64_t)row * p.N + col0);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const float4 a = p0[q];
+            acc[4 * q] = __float_as_uint(a.x), acc[4 * q + 1] = __float_as_uint(a.y);
+            acc[4 * q + 2] = __float_as_uint(a.z), acc[4 * q + 3] = __float_as_uint(a.w);
+        }
         for (int s = 1; s < S; ++s) {
-            const float4* ps = reinterpret_cast<const float4*>(partials + ((int64_t)s * M_cap + row) * N + col0);
-            a = ps[0], b = ps[1];
-            v[0] += a.x, v[1] += a.y, v[2] += a.z, v[3] += a.w, v[4] += b.x, v[5] += b.y, v[6] += b.z, v[7] += b.w;
-        }
-        if (bias != nullptr) {
-            const uint4 w = *reinterpret_cast<const uint4*>(bias + col0);
-            const uint32_t* ww = reinterpret_cast<const uint32_t*>(&w);
+            const float4* ps = reinterpret_cast<const float4*>(partials + ((int64_t)s * p.M_cap + row) * p.N + col0);
 #pragma unroll
-            for (int h = 0; h < 4; ++h) {
-                const float2 f = unpack2<T>(ww[h]);
-                v[2 * h] += f.x;
-                v[2 * h + 1] += f.y;
+            for (int q = 0; q < 8; ++q) {
+                const float4 a = ps[q];
+                acc[4 * q] = __float_as_uint(__uint_as_float(acc[4 * q]) + a.x);
+                acc[4 * q + 1] = __float_as_uint(__uint_as_float(acc[4 * q + 1]) + a.y);
+                acc[4 * q + 2] = __float_as_uint(__uint_as_float(acc[4 * q + 2]) + a.z);
+                acc[4 * q + 3] = __float_as_uint(__uint_as_float(acc[4 * q + 3]) + a.w);
             }
         }
-        if (EPI == EPI_BIAS_GELU) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) v[j] = gelu_tanh ? gelu_tanh_fast(v[j]) : gelu_f(v[j], false);
-        }
-        const int64_t off = (int64_t)row * N + col0;
-        if (EPI == EPI_BIAS_RESIDUAL) {
-            const uint4 w = *reinterpret_cast<const uint4*>(residual + off);
-            const uint32_t* ww = reinterpret_cast<const uint32_t*>(&w);
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-                const float2 f = unpack2<T>(ww[h]);
-                v[2 * h] += f.x;
-                v[2 * h + 1] += f.y;
-            }
-        }
-        uint4 o;
-        o.x = pack2<T>(v[0], v[1]);
-        o.y = pack2<T>(v[2], v[3]);
-        o.z = pack2<T>(v[4], v[5]);
-        o.w = pack2<T>(v[6], v[7]);
-        *reinterpret_cast<uint4*>(out + off) = o;
+        constexpr int NV = Epi<EPI>::RES_VECS > 0 ? Epi<EPI>::RES_VECS : 1;
+        uint4 res[NV];
+        load_residual32<T, EPI>(p, row, col0, true, res);
+        const float2 fs = Epi<EPI>::FOLD ? p.fold_stats[row] : make_float2(0.0f, 0.0f);
+        epilogue_store32<T, EPI>(acc, res, p, row, row, col0, fs);
     }
 }
 
@@ -613,7 +701,7 @@ template <typename T, int EPI, int MT>
 __global__ void __launch_bounds__(PairCfg<MT>::THREADS, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmR,
-                    const TcParams p) {
+                    const __grid_constant__ CUtensorMap tmL, const TcParams p) {
     using C = PairCfg<MT>;
     constexpr int NST = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
@@ -687,8 +775,9 @@ __global__ void __launch_bounds__(PairCfg<MT>::THREADS, 1)
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
-        tma_prefetch_desc(&tmO);
-        if (EPI == EPI_BIAS_RESIDUAL) tma_prefetch_desc(&tmR);
+        if (!Epi<EPI>::OUT_F32) tma_prefetch_desc(&tmO);
+        if (Epi<EPI>::RES_T) tma_prefetch_desc(&tmR);
+        if (Epi<EPI>::FOLD && p.lo != nullptr) tma_prefetch_desc(&tmL);
     }
     if (warp == 2) {
         tmem_alloc_pair(tmem_slot, TMEM_COLS);
@@ -846,7 +935,7 @@ __global__ void __launch_bounds__(PairCfg<MT>::THREADS, 1)
                     out_base = b * p.scatter_pad_len + (row_base - start);
                 }
                 if (box) {
-                    ok = drain_256_staged<T, EPI>(tbase, p, &tmO, &tmR, sbuf, rb, rpar, row_base, out_base, n * PBN,
+                    ok = drain_256_staged<T, EPI>(tbase, p, &tmO, &tmR, &tmL, sbuf, rb, rpar, row_base, out_base, n * PBN,
                                                   tempty_cluster, abort_flag);
                     handed_back = ok;
                 } else {
@@ -924,14 +1013,27 @@ static bool use_single_cta(const GemmArgs& a) { return a.M_cap <= TBM; }
 
 bool gemm_tc_scatter_ok(const GemmArgs& a) { return gemm_tc_supported(a) && !use_single_cta(a); }
 
+// The epilogues the layer uses: the folded LayerNorm (QKV), bias + GELU (FFN1), bias +
+// residual into fp32 (out-projection), bias + fp32 residual (FFN2).
+static bool tc_epilogue(int epi) {
+    return epi == EPI_LN_FOLD || epi == EPI_BIAS_GELU || epi == EPI_RES_OUT32 || epi == EPI_RES32;
+}
+
 bool gemm_tc_supported(const GemmArgs& a) {
     if (a.dtype != ENERGON_F16 && a.dtype != ENERGON_BF16) return false;
+    if (!tc_epilogue(a.epilogue)) return false;
     if (a.K < TBK || a.K % TBK != 0 || a.N < TBN || a.N % TBN != 0) return false;
     if (a.M_cap <= 0 || a.A_rows < PBM || a.A_rows % PBM != 0 || a.A_rows < a.M_cap) return false;
+    const bool res = a.epilogue == EPI_RES_OUT32 || a.epilogue == EPI_RES32;
+    if (res && a.residual == nullptr) return false;
+    if (a.epilogue == EPI_LN_FOLD) {
+        if (!a.fold_stats || !a.fold_c || !a.fold_d) return false;
+        if (a.lo != nullptr && (a.lo_cols <= 0 || a.lo_cols % TBN != 0 || a.lo_cols > a.N)) return false;
+    }
     const uintptr_t al = (uintptr_t)a.A | (uintptr_t)a.W | (uintptr_t)a.out | (uintptr_t)a.bias |
-                         (uintptr_t)(a.epilogue == EPI_BIAS_RESIDUAL ? a.residual : nullptr);
+                         (uintptr_t)(res ? a.residual : nullptr) | (uintptr_t)a.lo | (uintptr_t)a.fold_c |
+                         (uintptr_t)a.fold_d | (uintptr_t)a.fold_stats;
     if (al % 16 != 0) return false;
-    if (a.epilogue == EPI_BIAS_RESIDUAL && a.residual == nullptr) return false;
     return encode_fn() != nullptr;
 }
 
@@ -946,7 +1048,8 @@ static cudaError_t tc_launch(const CUtensorMap& ta, const CUtensorMap& tb, const
 
 template <typename T, int EPI, int MT>
 static cudaError_t tc2_launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to,
-                              const CUtensorMap& tr, const TcParams& p, int pairs, cudaStream_t st) {
+                              const CUtensorMap& tr, const CUtensorMap& tl, const TcParams& p, int pairs,
+                              cudaStream_t st) {
     using C = PairCfg<MT>;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -979,19 +1082,44 @@ static cudaError_t tc2_launch(const CUtensorMap& ta, const CUtensorMap& tb, cons
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<T, EPI, MT>, ta, tb, to, tr, p);
+    return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<T, EPI, MT>, ta, tb, to, tr, tl, p);
 }
 
 template <typename T, int MT>
 static cudaError_t tc2_dispatch(int epi, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to,
-                                const CUtensorMap& tr, const TcParams& p, int pairs, cudaStream_t st) {
+                                const CUtensorMap& tr, const CUtensorMap& tl, const TcParams& p, int pairs,
+                                cudaStream_t st) {
     switch (epi) {
-    case EPI_BIAS: return tc2_launch<T, EPI_BIAS, MT>(ta, tb, to, tr, p, pairs, st);
-    case EPI_BIAS_GELU: return tc2_launch<T, EPI_BIAS_GELU, MT>(ta, tb, to, tr, p, pairs, st);
-    default: return tc2_launch<T, EPI_BIAS_RESIDUAL, MT>(ta, tb, to, tr, p, pairs, st);
+    case EPI_LN_FOLD: return tc2_launch<T, EPI_LN_FOLD, MT>(ta, tb, to, tr, tl, p, pairs, st);
+    case EPI_BIAS_GELU: return tc2_launch<T, EPI_BIAS_GELU, MT>(ta, tb, to, tr, tl, p, pairs, st);
+    case EPI_RES_OUT32: return tc2_launch<T, EPI_RES_OUT32, MT>(ta, tb, to, tr, tl, p, pairs, st);
+    default: return tc2_launch<T, EPI_RES32, MT>(ta, tb, to, tr, tl, p, pairs, st);
     }
 }
 
+template <typename T>
+static cudaError_t single_dispatch(int epi, const CUtensorMap& ta, const CUtensorMap& tb, const TcParams& p,
+                                   int grid, int fgrid, cudaStream_t st) {
+    cudaError_t e;
+    switch (epi) {
+    case EPI_LN_FOLD: e = tc_launch<T, EPI_LN_FOLD>(ta, tb, p, grid, st); break;
+    case EPI_BIAS_GELU: e = tc_launch<T, EPI_BIAS_GELU>(ta, tb, p, grid, st); break;
+    case EPI_RES_OUT32: e = tc_launch<T, EPI_RES_OUT32>(ta, tb, p, grid, st); break;
+    default: e = tc_launch<T, EPI_RES32>(ta, tb, p, grid, st); break;
+    }
+    if (e != cudaSuccess || p.k_splits == 1) return e;
+    switch (epi) {
+    case EPI_LN_FOLD: splitk_finish_kernel<T, EPI_LN_FOLD><<<fgrid, 256, 0, st>>>(p.partials, p.k_splits, p); break;
+    case EPI_BIAS_GELU:
+        splitk_finish_kernel<T, EPI_BIAS_GELU><<<fgrid, 256, 0, st>>>(p.partials, p.k_splits, p);
+        break;
+    case EPI_RES_OUT32:
+        splitk_finish_kernel<T, EPI_RES_OUT32><<<fgrid, 256, 0, st>>>(p.partials, p.k_splits, p);
+        break;
+    default: splitk_finish_kernel<T, EPI_RES32><<<fgrid, 256, 0, st>>>(p.partials, p.k_splits, p); break;
+    }
+    return cudaGetLastError();
+}
 
 cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st, char* err, size_t errlen) {
     const bool single = use_single_cta(a);
@@ -1018,9 +1146,15 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st, char* err, size_t
     p.scatter_cu = a.scatter_cu;
     p.scatter_batch = a.scatter_batch;
     p.scatter_pad_len = a.scatter_pad_len;
+    p.fold_stats = a.fold_stats;
+    p.fold_c = a.fold_c;
+    p.fold_d = a.fold_d;
+    p.lo = a.epilogue == EPI_LN_FOLD ? a.lo : nullptr;
+    p.lo_cols = p.lo ? a.lo_cols : 0;
     const bool bf = a.dtype == ENERGON_BF16;
-    if (single && a.scatter_cu != nullptr) {
-        if (err) snprintf(err, errlen, "scattering epilogue needs the CTA-pair path (more than %d rows)", TBM);
+    if (a.scatter_cu != nullptr && (single || a.epilogue == EPI_RES_OUT32 || a.epilogue == EPI_LN_FOLD)) {
+        if (err) snprintf(err, errlen, "a scattering epilogue needs the CTA-pair path (more than %d rows) and a "
+                                       "16-bit output without low halves", TBM);
         return cudaErrorInvalidValue;
     }
     if (!single) {
@@ -1032,23 +1166,33 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st, char* err, size_t
         p.group_m = 1;
         const int64_t tiles_cap = (int64_t)num_m_cap * num_n;
         const int pairs = (int)(tiles_cap < device_sm_count() / 2 ? tiles_cap : device_sm_count() / 2);
-        // Output (and residual) as 32 x 32 boxes, 64-byte swizzle: the epilogue's staged
-        // stores and residual loads.  Only boxes of rows below the live row count are
-        // ever copied, so the maps may span the whole buffer capacity.
-        CUtensorMap to, tr;
+        // Output, residual and low halves as 32 x 32 boxes, 64-byte swizzle: the epilogue's
+        // staged stores and residual loads.  Only boxes of rows below the live row count are
+        // ever copied, so the maps may span the whole buffer capacity.  A map the epilogue
+        // does not use is a copy of one that exists.
+        CUtensorMap to, tr, tl;
         const int64_t out_rows = a.scatter_cu ? (int64_t)a.scatter_batch * a.scatter_pad_len : a.M_cap;
-        CUresult r3 = make_tmap_io(&to, a.dtype, a.out, a.N, out_rows);
-        CUresult r4 = a.epilogue == EPI_BIAS_RESIDUAL ? make_tmap_io(&tr, a.dtype, a.residual, a.N, a.M_cap) : r3;
-        if (a.epilogue != EPI_BIAS_RESIDUAL) tr = to;
-        if (r3 != CUDA_SUCCESS || r4 != CUDA_SUCCESS) {
-            if (err) snprintf(err, errlen, "cuTensorMapEncodeTiled failed (out: %d, residual: %d)", (int)r3, (int)r4);
+        CUresult r3 = CUDA_SUCCESS, r4 = CUDA_SUCCESS, r5 = CUDA_SUCCESS;
+        if (a.epilogue == EPI_RES_OUT32) {
+            r4 = make_tmap_io(&tr, a.dtype, a.residual, a.N, a.M_cap);
+            to = tr;
+        } else {
+            r3 = make_tmap_io(&to, a.dtype, a.out, a.N, out_rows);
+            tr = to;
+        }
+        if (p.lo != nullptr) r5 = make_tmap_io(&tl, a.dtype, p.lo, p.lo_cols, a.M_cap);
+        else tl = to;
+        if (r3 != CUDA_SUCCESS || r4 != CUDA_SUCCESS || r5 != CUDA_SUCCESS) {
+            if (err)
+                snprintf(err, errlen, "cuTensorMapEncodeTiled failed (out: %d, residual: %d, low halves: %d)", (int)r3,
+                         (int)r4, (int)r5);
             return cudaErrorInvalidValue;
         }
         if (mt == 2)
-            return bf ? tc2_dispatch<__nv_bfloat16, 2>(a.epilogue, ta, tb, to, tr, p, pairs, st)
-                      : tc2_dispatch<__half, 2>(a.epilogue, ta, tb, to, tr, p, pairs, st);
-        return bf ? tc2_dispatch<__nv_bfloat16, 1>(a.epilogue, ta, tb, to, tr, p, pairs, st)
-                  : tc2_dispatch<__half, 1>(a.epilogue, ta, tb, to, tr, p, pairs, st);
+            return bf ? tc2_dispatch<__nv_bfloat16, 2>(a.epilogue, ta, tb, to, tr, tl, p, pairs, st)
+                      : tc2_dispatch<__half, 2>(a.epilogue, ta, tb, to, tr, tl, p, pairs, st);
+        return bf ? tc2_dispatch<__nv_bfloat16, 1>(a.epilogue, ta, tb, to, tr, tl, p, pairs, st)
+                  : tc2_dispatch<__half, 1>(a.epilogue, ta, tb, to, tr, tl, p, pairs, st);
     }
     const int num_m_cap = (a.M_cap + TBM - 1) / TBM, num_n = a.N / TBN;
     // Rows of A kept hot per raster group: about 48 MiB of the 126 MB L2.
@@ -1075,39 +1219,10 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st, char* err, size_t
     p.partials = a.partials;
     const int64_t units = tiles * S;
     const int grid = (int)(units < sms ? units : sms);
-    cudaError_t e;
-    switch (a.epilogue) {
-    case EPI_BIAS:
-        e = bf ? tc_launch<__nv_bfloat16, EPI_BIAS>(ta, tb, p, grid, st) : tc_launch<__half, EPI_BIAS>(ta, tb, p, grid, st);
-        break;
-    case EPI_BIAS_GELU:
-        e = bf ? tc_launch<__nv_bfloat16, EPI_BIAS_GELU>(ta, tb, p, grid, st)
-               : tc_launch<__half, EPI_BIAS_GELU>(ta, tb, p, grid, st);
-        break;
-    default:
-        e = bf ? tc_launch<__nv_bfloat16, EPI_BIAS_RESIDUAL>(ta, tb, p, grid, st)
-               : tc_launch<__half, EPI_BIAS_RESIDUAL>(ta, tb, p, grid, st);
-        break;
-    }
-    if (e != cudaSuccess || S == 1) return e;
-    const int64_t work = (int64_t)a.M_cap * (a.N / 8);
+    const int64_t work = (int64_t)a.M_cap * (a.N / 32);
     const int fgrid = (int)((work + 255) / 256 < 4 * sms ? (work + 255) / 256 : 4 * sms);
-#define FINISH(TT, EE)                                                                                              \
-    splitk_finish_kernel<TT, EE><<<fgrid, 256, 0, st>>>(a.partials, S, a.M_cap, a.d_rows, a.N, (const TT*)a.bias, \
-                                                        (const TT*)a.residual, (TT*)a.out, a.gelu_tanh, a.status)
-    switch (a.epilogue) {
-    case EPI_BIAS:
-        if (bf) FINISH(__nv_bfloat16, EPI_BIAS); else FINISH(__half, EPI_BIAS);
-        break;
-    case EPI_BIAS_GELU:
-        if (bf) FINISH(__nv_bfloat16, EPI_BIAS_GELU); else FINISH(__half, EPI_BIAS_GELU);
-        break;
-    default:
-        if (bf) FINISH(__nv_bfloat16, EPI_BIAS_RESIDUAL); else FINISH(__half, EPI_BIAS_RESIDUAL);
-        break;
-    }
-#undef FINISH
-    return cudaGetLastError();
+    return bf ? single_dispatch<__nv_bfloat16>(a.epilogue, ta, tb, p, grid, fgrid, st)
+              : single_dispatch<__half>(a.epilogue, ta, tb, p, grid, fgrid, st);
 }
 
 }  // namespace energon

@@ -51,13 +51,32 @@ struct LnGather {
     int batch = 0, pad_len = 0;
     void* copy = nullptr;
 };
-// LayerNorm over rows [0, min(*d_rows, rows_cap)) of x [rows_cap, H] -> y.
+// LayerNorm over rows [0, min(*d_rows, rows_cap)) of x [rows_cap, H] -> y.  x_f32: the
+// input rows are fp32 (the residual after attention), y is of the storage type.
 cudaError_t launch_layernorm(int dtype, const void* x, const void* g, const void* b, void* y, const int32_t* d_rows,
                              int rows_cap, int H, float eps, const int32_t* status, cudaStream_t st,
-                             const LnGather& gth = LnGather());
+                             const LnGather& gth = LnGather(), bool x_f32 = false);
+
+// LayerNorm folded into the GEMM that follows it.  For each row r of x (storage type):
+//   u[r][k] = x[r][k] * g[k] rounded to the storage type (exact when g is 1),
+//   stats[r] = (rstd_r, mean_r * rstd_r) in fp32,
+// so that LN(x) W^T + b = rstd_r (u W^T) - mean_r rstd_r c + d with the vectors of
+// launch_ln_fold_weights.  Gather form as in launch_layernorm.
+cudaError_t launch_ln_fold(int dtype, const void* x, const void* g, void* u, float2* stats, const int32_t* d_rows,
+                           int rows_cap, int H, float eps, const int32_t* status, cudaStream_t st,
+                           const LnGather& gth = LnGather());
+// c[n] = sum_k g[k] W[n][k], d[n] = bias[n] + sum_k beta[k] W[n][k] (fp32) for W [N, K].
+cudaError_t launch_ln_fold_weights(int dtype, const void* W, const void* g, const void* beta, const void* bias,
+                                   int N, int K, float* c, float* d, const int32_t* status, cudaStream_t st);
 
 // Epilogue variants of the GEMM y = A W^T + bias (+ GELU) (+ residual).
-enum Epilogue { EPI_BIAS = 0, EPI_BIAS_GELU = 1, EPI_BIAS_RESIDUAL = 2 };
+//   EPI_LN_FOLD: y = rstd_r acc - (mean rstd)_r c[n] + d[n] (the folded LayerNorm,
+//     see launch_ln_fold); columns below lo_cols also store y - round(y), rounded,
+//     to `lo` (the low half of a two-term 16-bit value).
+//   EPI_RES_OUT32: y = acc + bias + residual (storage type), stored as fp32.
+//   EPI_RES32: y = acc + bias + residual (fp32), stored in the storage type.
+enum Epilogue { EPI_BIAS = 0, EPI_BIAS_GELU = 1, EPI_BIAS_RESIDUAL = 2, EPI_LN_FOLD = 3, EPI_RES_OUT32 = 4,
+                EPI_RES32 = 5 };
 
 struct GemmArgs {
     int dtype;                 // energon_dtype
@@ -79,6 +98,12 @@ struct GemmArgs {
     // row b * scatter_pad_len + r - scatter_cu[b] of out [scatter_batch, scatter_pad_len, N].
     const int32_t* scatter_cu = nullptr;
     int scatter_batch = 0, scatter_pad_len = 0;
+    // EPI_LN_FOLD: per-row (rstd, mean * rstd), per-column c and d, and the low halves
+    const float2* fold_stats = nullptr;
+    const float* fold_c = nullptr;
+    const float* fold_d = nullptr;
+    void* lo = nullptr;        // [M_cap, lo_cols] or null
+    int lo_cols = 0;
 };
 
 // True when the tcgen05 path can run this GEMM (16-bit types, alignment, tile multiples).
@@ -91,11 +116,16 @@ cudaError_t launch_gemm_simt(const GemmArgs& a, cudaStream_t st);
 // Causal attention within each sequence: qkv [rows, 3H] -> o [rows, H].  The
 // tensor-core kernel runs for 16-bit types with head_dim 128 (qkv_rows: rows
 // allocated in qkv, the extent of its tensor map); otherwise the CUDA-core one.
-cudaError_t launch_attention(int dtype, const void* qkv, void* o, const int32_t* cu, int batch, int max_len, int H,
-                             int n_heads, int qkv_rows, int32_t* status, uint64_t timeout_ns, cudaStream_t st);
-bool attention_tc_supported(int dtype, int H, int n_heads, const void* qkv, const void* o, int qkv_rows);
-cudaError_t launch_attention_tc(int dtype, const void* qkv, void* o, const int32_t* cu, int batch, int max_len, int H,
-                                int n_heads, int qkv_rows, int32_t* status, uint64_t timeout_ns, cudaStream_t st);
+// qk_lo [rows, 2H] (optional): the low halves of Q | K, so that q = hi + lo to about twice
+// the storage type's precision; the scores then use both halves.
+cudaError_t launch_attention(int dtype, const void* qkv, const void* qk_lo, void* o, const int32_t* cu, int batch,
+                             int max_len, int H, int n_heads, int qkv_rows, int32_t* status, uint64_t timeout_ns,
+                             cudaStream_t st);
+bool attention_tc_supported(int dtype, int H, int n_heads, const void* qkv, const void* qk_lo, const void* o,
+                            int qkv_rows);
+cudaError_t launch_attention_tc(int dtype, const void* qkv, const void* qk_lo, void* o, const int32_t* cu, int batch,
+                                int max_len, int H, int n_heads, int qkv_rows, int32_t* status, uint64_t timeout_ns,
+                                cudaStream_t st);
 
 // The binary version (major * 10 + minor) the runtime reports for the library's kernels.
 cudaError_t kernel_binary_version(int* version);

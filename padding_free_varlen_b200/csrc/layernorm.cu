@@ -1,34 +1,91 @@
 // LayerNorm of the pre-LN GPT layer: y = (x - mean) / sqrt(var + eps) * g + b,
-// biased variance, statistics in fp32, output rounded to the storage type.
-// (The normalisation of the bias + residual + LayerNorm step in the QbitAI
-// article's FasterTransformer excerpt, section "易用性", placed before each
-// sub-layer as in GPT-2/3.)
+// biased variance, statistics in fp32.  (The normalisation of the bias +
+// residual + LayerNorm step in the QbitAI article's FasterTransformer excerpt,
+// section "易用性", placed before each sub-layer as in GPT-2/3.)
 //
-// One thread block per row (grid-stride over the device-side row count).  For
-// 16-bit rows of up to 16384 elements each thread keeps its slice in registers
-// as 16-byte vectors, so the row is read from HBM once and written once.
+// Two forms:
+//  - ln_rows_kernel: the LayerNorm before the MLP.  Its input is the fp32
+//    residual after attention, its output (the FFN1 operand) the storage type.
+//    One thread block per row; each thread keeps its slice of the row in
+//    registers, so the row is read from HBM once and written once.
+//  - ln_fold_kernel: the LayerNorm before the QKV projection, folded into that
+//    GEMM.  It writes u = x * g (rounded to the storage type: exact when g is 1)
+//    and the row statistics (rstd, mean * rstd); the GEMM's epilogue finishes
+//    LN(x) W^T + b = rstd (u W^T) - mean rstd c + d with c = W g, d = b + W beta
+//    (ln_fold_weights_kernel).  The tensor cores then see the layer input
+//    itself instead of a rounded normalisation of it, which the attention
+//    scores that follow are sensitive to.
+//    Gather form (transpose_padding_remove fused into the first LayerNorm):
+//    packed row r reads padded row (b, r - cu[b]) of a [batch, pad_len, H]
+//    tensor and also writes that raw row to `copy` (the packed residual stream),
+//    so the padded input is read once for both.
 //
-// Gather form (transpose_padding_remove fused into the first LayerNorm): packed
-// row r reads padded row (b, r - cu[b]) of a [batch, pad_len, H] tensor and also
-// writes that raw row to `copy` (the packed residual stream), so the padded input
-// is read once for both.
+// Row statistics use sums shifted by the row's first element, s1 = sum (x - x0)
+// and s2 = sum (x - x0)^2 (one block reduction of the pair): mean = x0 + s1 / H,
+// var = s2 / H - (s1 / H)^2.  The shift keeps the subtraction benign when the
+// mean is large against the spread.
 #include "common.cuh"
 #include "internal.h"
 
 namespace energon {
 
-// Sum over the block; every thread gets the result.  `red` holds 32 floats.
-__device__ __forceinline__ float block_sum(float v, float* red) {
+// N elements of T in one aligned vector (16 bytes for the vector paths).
+template <typename T, int N>
+struct alignas(N * sizeof(T)) Pack {
+    T v[N];
+};
+
+template <typename T, int N>
+__device__ __forceinline__ void load_f(const T* p, float* f) {
+    const Pack<T, N> pk = *reinterpret_cast<const Pack<T, N>*>(p);
+#pragma unroll
+    for (int i = 0; i < N; ++i) f[i] = to_f(pk.v[i]);
+}
+template <typename T, int N>
+__device__ __forceinline__ void load_f_ldg(const T* p, float* f) {
+    Pack<T, N> pk;
+    if constexpr (sizeof(Pack<T, N>) == 16) {
+        const uint4 w = __ldg(reinterpret_cast<const uint4*>(p));
+        pk = *reinterpret_cast<const Pack<T, N>*>(&w);
+    } else {
+        pk = *reinterpret_cast<const Pack<T, N>*>(p);
+    }
+#pragma unroll
+    for (int i = 0; i < N; ++i) f[i] = to_f(pk.v[i]);
+}
+template <typename T, int N>
+__device__ __forceinline__ void store_f(T* p, const float* f) {
+    Pack<T, N> pk;
+#pragma unroll
+    for (int i = 0; i < N; ++i) pk.v[i] = from_f<T>(f[i]);
+    *reinterpret_cast<Pack<T, N>*>(p) = pk;
+}
+
+// Sum of a float pair over the block; every thread gets the result.  `red` holds 32 pairs.
+__device__ __forceinline__ float2 block_sum2(float2 v, float2* red) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    __syncthreads();  // red may still be read from a previous call
+    for (int o = 16; o > 0; o >>= 1) {
+        v.x += __shfl_xor_sync(0xffffffffu, v.x, o);
+        v.y += __shfl_xor_sync(0xffffffffu, v.y, o);
+    }
+    __syncthreads();  // red may still be read from the previous row
     if (lane == 0) red[warp] = v;
     __syncthreads();
-    float t = lane < nw ? red[lane] : 0.0f;
+    float2 t = lane < nw ? red[lane] : make_float2(0.0f, 0.0f);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    for (int o = 16; o > 0; o >>= 1) {
+        t.x += __shfl_xor_sync(0xffffffffu, t.x, o);
+        t.y += __shfl_xor_sync(0xffffffffu, t.y, o);
+    }
     return t;
+}
+
+// (mean, 1 / sqrt(var + eps)) from the shifted sums of a row of H elements.
+__device__ __forceinline__ float2 row_stats(float x0, float2 s, int H, float eps) {
+    const float m1 = s.x / H;
+    const float var = fmaxf(s.y / H - m1 * m1, 0.0f);
+    return make_float2(x0 + m1, rsqrtf(var + eps));
 }
 
 // Source row of packed row r: itself, or (gather) padded row (b, r - cu[b]); -1 if
@@ -40,107 +97,179 @@ __device__ __forceinline__ int64_t ln_src_row(const LnGather& gth, int r) {
     return (s >= 0 && s < gth.pad_len) ? (int64_t)b * gth.pad_len + s : -1;
 }
 
-template <typename T>
-__global__ void __launch_bounds__(256) ln_generic_kernel(const T* __restrict__ x, const T* __restrict__ g,
-                                                         const T* __restrict__ bb, T* __restrict__ y,
-                                                         const int32_t* d_rows, int rows_cap, int H, float eps,
-                                                         const int32_t* status, LnGather gth) {
-    __shared__ float red[32];
+// ------------------------------------------------------------------ LayerNorm (row in registers)
+
+// Tin: input element type (the storage type, or float for the fp32 residual), Tout: the
+// storage type.  N = elements per 16-byte input vector; VPT vectors per thread (the row
+// has H / N vectors, H % N == 0, at most 256 * VPT of them).
+template <typename Tin, typename Tout, int VPT>
+__global__ void __launch_bounds__(256) ln_rows_kernel(const Tin* __restrict__ x, const Tout* __restrict__ g,
+                                                      const Tout* __restrict__ bb, Tout* __restrict__ y,
+                                                      const int32_t* d_rows, int rows_cap, int H, float eps,
+                                                      const int32_t* status) {
+    constexpr int N = 16 / sizeof(Tin);
+    __shared__ float2 red[32];
     if (status_bad(status)) return;
     const int rows = min(*d_rows, rows_cap);
+    const int nvec = H / N;
+    for (int r = blockIdx.x; r < rows; r += gridDim.x) {
+        const Tin* xr = x + (int64_t)r * H;
+        const float x0 = to_f(xr[0]);
+        float f[VPT][N];
+        float2 s = make_float2(0.0f, 0.0f);
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            const int idx = i * blockDim.x + threadIdx.x;
+            if (idx < nvec) {
+                load_f<Tin, N>(xr + (int64_t)idx * N, f[i]);
+#pragma unroll
+                for (int j = 0; j < N; ++j) {
+                    const float d = f[i][j] - x0;
+                    s.x += d;
+                    s.y = fmaf(d, d, s.y);
+                }
+            }
+        }
+        const float2 mi = row_stats(x0, block_sum2(s, red), H, eps);
+        Tout* yr = y + (int64_t)r * H;
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            const int idx = i * blockDim.x + threadIdx.x;
+            if (idx < nvec) {
+                float gv[N], bv[N], o[N];
+                load_f_ldg<Tout, N>(g + (int64_t)idx * N, gv);
+                load_f_ldg<Tout, N>(bb + (int64_t)idx * N, bv);
+#pragma unroll
+                for (int j = 0; j < N; ++j) o[j] = (f[i][j] - mi.x) * mi.y * gv[j] + bv[j];
+                store_f<Tout, N>(yr + (int64_t)idx * N, o);
+            }
+        }
+    }
+}
+
+// Any H, any alignment: three passes over the row (L1/L2 serve the repeats).
+template <typename Tin, typename Tout>
+__global__ void __launch_bounds__(256) ln_rows_generic_kernel(const Tin* __restrict__ x, const Tout* __restrict__ g,
+                                                              const Tout* __restrict__ bb, Tout* __restrict__ y,
+                                                              const int32_t* d_rows, int rows_cap, int H, float eps,
+                                                              const int32_t* status) {
+    __shared__ float2 red[32];
+    if (status_bad(status)) return;
+    const int rows = min(*d_rows, rows_cap);
+    for (int r = blockIdx.x; r < rows; r += gridDim.x) {
+        const Tin* xr = x + (int64_t)r * H;
+        const float x0 = to_f(xr[0]);
+        float2 s = make_float2(0.0f, 0.0f);
+        for (int k = threadIdx.x; k < H; k += blockDim.x) {
+            const float d = to_f(xr[k]) - x0;
+            s.x += d;
+            s.y = fmaf(d, d, s.y);
+        }
+        const float2 mi = row_stats(x0, block_sum2(s, red), H, eps);
+        Tout* yr = y + (int64_t)r * H;
+        for (int k = threadIdx.x; k < H; k += blockDim.x)
+            yr[k] = from_f<Tout>((to_f(xr[k]) - mi.x) * mi.y * to_f(g[k]) + to_f(bb[k]));
+    }
+}
+
+// ------------------------------------------------------------------ LayerNorm folded into the GEMM
+
+// u = x * g, stats = (rstd, mean * rstd); N elements per step (16-byte vectors when VEC).
+template <typename T, bool VEC>
+__global__ void __launch_bounds__(256) ln_fold_kernel(const T* __restrict__ x, const T* __restrict__ g,
+                                                      T* __restrict__ u, float2* __restrict__ stats,
+                                                      const int32_t* d_rows, int rows_cap, int H, float eps,
+                                                      const int32_t* status, LnGather gth) {
+    constexpr int N = VEC ? 16 / sizeof(T) : 1;
+    __shared__ float2 red[32];
+    if (status_bad(status)) return;
+    const int rows = min(*d_rows, rows_cap);
+    const int nvec = H / N;
+    T* copy = static_cast<T*>(gth.copy);
     for (int r = blockIdx.x; r < rows; r += gridDim.x) {
         const int64_t src = ln_src_row(gth, r);
         if (src < 0) continue;
         const T* xr = x + src * H;
-        if (gth.copy != nullptr) {
-            T* cr = static_cast<T*>(gth.copy) + (int64_t)r * H;
-            for (int k = threadIdx.x; k < H; k += blockDim.x) cr[k] = xr[k];
+        T* ur = u + (int64_t)r * H;
+        T* cr = copy ? copy + (int64_t)r * H : nullptr;
+        const float x0 = to_f(xr[0]);
+        float2 s = make_float2(0.0f, 0.0f);
+#pragma unroll 4
+        for (int idx = threadIdx.x; idx < nvec; idx += blockDim.x) {
+            const int64_t e = (int64_t)idx * N;
+            const Pack<T, N> xv = *reinterpret_cast<const Pack<T, N>*>(xr + e);
+            if (cr) *reinterpret_cast<Pack<T, N>*>(cr + e) = xv;
+            float gv[N], o[N];
+            load_f_ldg<T, N>(g + e, gv);
+#pragma unroll
+            for (int j = 0; j < N; ++j) {
+                const float v = to_f(xv.v[j]);
+                const float d = v - x0;
+                s.x += d;
+                s.y = fmaf(d, d, s.y);
+                o[j] = v * gv[j];
+            }
+            store_f<T, N>(ur + e, o);
         }
-        float s = 0.0f;
-        for (int k = threadIdx.x; k < H; k += blockDim.x) s += to_f(xr[k]);
-        const float mean = block_sum(s, red) / H;
-        float q = 0.0f;
-        for (int k = threadIdx.x; k < H; k += blockDim.x) {
-            float d = to_f(xr[k]) - mean;
-            q += d * d;
-        }
-        const float var = block_sum(q, red) / H;
-        const float inv = 1.0f / sqrtf(var + eps);
-        T* yr = y + (int64_t)r * H;
-        for (int k = threadIdx.x; k < H; k += blockDim.x)
-            yr[k] = from_f<T>((to_f(xr[k]) - mean) * inv * to_f(g[k]) + to_f(bb[k]));
+        const float2 mi = row_stats(x0, block_sum2(s, red), H, eps);
+        if (threadIdx.x == 0) stats[r] = make_float2(mi.y, mi.x * mi.y);
     }
 }
 
-// 16-bit types, H % 8 == 0, H / 8 <= 256 * VPT, 16-byte aligned pointers.
-template <typename T, int VPT>
-__global__ void __launch_bounds__(256) ln_vec_kernel(const T* __restrict__ x, const T* __restrict__ g,
-                                                     const T* __restrict__ bb, T* __restrict__ y,
-                                                     const int32_t* d_rows, int rows_cap, int H, float eps,
-                                                     const int32_t* status, LnGather gth) {
-    __shared__ float red[32];
+// c[n] = sum_k g[k] W[n][k], d[n] = bias[n] + sum_k beta[k] W[n][k].  Each warp owns RPW
+// consecutive rows of W and walks K once, with g and beta loaded once per step for all
+// of its rows; lane-strided partial sums, then a fixed shuffle tree (deterministic).
+template <typename T, bool VEC, int RPW>
+__global__ void __launch_bounds__(256) ln_fold_weights_kernel(const T* __restrict__ W, const T* __restrict__ g,
+                                                              const T* __restrict__ beta, const T* __restrict__ bias,
+                                                              int Nrows, int K, float* __restrict__ c,
+                                                              float* __restrict__ d, const int32_t* status) {
+    constexpr int N = VEC ? 16 / sizeof(T) : 1;
     if (status_bad(status)) return;
-    const int rows = min(*d_rows, rows_cap);
-    const int nvec = H / 8;
-    uint4* copy = static_cast<uint4*>(gth.copy);
-    for (int r = blockIdx.x; r < rows; r += gridDim.x) {
-        const int64_t src = ln_src_row(gth, r);
-        if (src < 0) continue;
-        const uint4* xr = reinterpret_cast<const uint4*>(x + src * H);
-        uint4 v[VPT];
-        float s = 0.0f;
+    const int lane = threadIdx.x & 31;
+    const int n0 = (blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * RPW;
+    if (n0 >= Nrows) return;
+    float ac[RPW], ad[RPW];
 #pragma unroll
-        for (int i = 0; i < VPT; ++i) {
-            const int idx = i * blockDim.x + threadIdx.x;
-            if (idx < nvec) {
-                v[i] = xr[idx];
-                if (copy != nullptr) copy[(int64_t)r * nvec + idx] = v[i];
-                const uint32_t* w = reinterpret_cast<const uint32_t*>(&v[i]);
+    for (int i = 0; i < RPW; ++i) ac[i] = ad[i] = 0.0f;
+    const int nvec = K / N;
+    for (int idx = lane; idx < nvec; idx += 32) {
+        const int64_t e = (int64_t)idx * N;
+        float gv[N], bv[N];
+        load_f_ldg<T, N>(g + e, gv);
+        load_f_ldg<T, N>(beta + e, bv);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    float2 f = unpack2<T>(w[j]);
-                    s += f.x + f.y;
+        for (int i = 0; i < RPW; ++i) {
+            if (n0 + i < Nrows) {
+                float wv[N];
+                load_f<T, N>(W + (int64_t)(n0 + i) * K + e, wv);
+#pragma unroll
+                for (int j = 0; j < N; ++j) {
+                    ac[i] = fmaf(gv[j], wv[j], ac[i]);
+                    ad[i] = fmaf(bv[j], wv[j], ad[i]);
                 }
-            }
-        }
-        const float mean = block_sum(s, red) / H;
-        float q = 0.0f;
-#pragma unroll
-        for (int i = 0; i < VPT; ++i) {
-            const int idx = i * blockDim.x + threadIdx.x;
-            if (idx < nvec) {
-                const uint32_t* w = reinterpret_cast<const uint32_t*>(&v[i]);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    float2 f = unpack2<T>(w[j]);
-                    q += (f.x - mean) * (f.x - mean) + (f.y - mean) * (f.y - mean);
-                }
-            }
-        }
-        const float var = block_sum(q, red) / H;
-        const float inv = 1.0f / sqrtf(var + eps);
-        uint4* yr = reinterpret_cast<uint4*>(y + (int64_t)r * H);
-#pragma unroll
-        for (int i = 0; i < VPT; ++i) {
-            const int idx = i * blockDim.x + threadIdx.x;
-            if (idx < nvec) {
-                const uint4 gv = __ldg(reinterpret_cast<const uint4*>(g) + idx);
-                const uint4 bv = __ldg(reinterpret_cast<const uint4*>(bb) + idx);
-                const uint32_t* w = reinterpret_cast<const uint32_t*>(&v[i]);
-                const uint32_t* gw = reinterpret_cast<const uint32_t*>(&gv);
-                const uint32_t* bw = reinterpret_cast<const uint32_t*>(&bv);
-                uint4 o;
-                uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    float2 f = unpack2<T>(w[j]), gf = unpack2<T>(gw[j]), bf = unpack2<T>(bw[j]);
-                    ow[j] = pack2<T>((f.x - mean) * inv * gf.x + bf.x, (f.y - mean) * inv * gf.y + bf.y);
-                }
-                yr[idx] = o;
             }
         }
     }
+#pragma unroll
+    for (int i = 0; i < RPW; ++i) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            ac[i] += __shfl_xor_sync(0xffffffffu, ac[i], o);
+            ad[i] += __shfl_xor_sync(0xffffffffu, ad[i], o);
+        }
+    }
+    if (lane == 0) {
+#pragma unroll
+        for (int i = 0; i < RPW; ++i)
+            if (n0 + i < Nrows) {
+                c[n0 + i] = ac[i];
+                d[n0 + i] = ad[i] + (bias ? to_f(bias[n0 + i]) : 0.0f);
+            }
+    }
 }
+
+// ------------------------------------------------------------------ host side
 
 // Blocks of `kernel` (256 threads) that fit on the GPU at once: the row loop then runs
 // in a single wave of blocks instead of leaving a second wave to start late.
@@ -156,57 +285,112 @@ static int resident_blocks(K kernel) {
     });
 }
 
-static int ln_grid(int rows_cap, int resident) {
+static int row_grid(int rows_cap, int resident) {
     return rows_cap < resident ? (rows_cap > 0 ? rows_cap : 1) : resident;
 }
 
-template <typename T>
-static cudaError_t ln_dispatch(const void* x, const void* g, const void* b, void* y, const int32_t* d_rows,
-                               int rows_cap, int H, float eps, const int32_t* status, const LnGather& gth,
-                               cudaStream_t st) {
-    const T *xp = (const T*)x, *gp = (const T*)g, *bp = (const T*)b;
-    T* yp = (T*)y;
-    const uintptr_t al = (uintptr_t)x | (uintptr_t)g | (uintptr_t)b | (uintptr_t)y | (uintptr_t)gth.copy;
-    const int nvec = H / 8;
-    const int vpt = (nvec + 255) / 256;
-    if (sizeof(T) == 2 && H % 8 == 0 && al % 16 == 0 && vpt >= 1 && vpt <= 8) {
-        switch (vpt) {
-#define LN_CASE(V)                                                                                      \
-    case V: {                                                                                           \
-        const int resident = resident_blocks(ln_vec_kernel<T, V>);                                      \
-        ln_vec_kernel<T, V><<<ln_grid(rows_cap, resident), 256, 0, st>>>(xp, gp, bp, yp, d_rows, rows_cap, H, \
-                                                                         eps, status, gth);             \
-        break;                                                                                          \
-    }
-            LN_CASE(1) LN_CASE(2) LN_CASE(3) LN_CASE(4) LN_CASE(5) LN_CASE(6) LN_CASE(7) LN_CASE(8)
-#undef LN_CASE
-        }
-    } else {
-        const int resident = resident_blocks(ln_generic_kernel<T>);
-        ln_generic_kernel<T><<<ln_grid(rows_cap, resident), 256, 0, st>>>(xp, gp, bp, yp, d_rows, rows_cap, H, eps,
-                                                                         status, gth);
-    }
-    return cudaGetLastError();
+template <typename Tin, typename Tout, int VPT>
+static void ln_rows_launch(const void* x, const void* g, const void* b, void* y, const int32_t* d_rows, int rows_cap,
+                           int H, float eps, const int32_t* status, cudaStream_t st) {
+    auto k = ln_rows_kernel<Tin, Tout, VPT>;
+    k<<<row_grid(rows_cap, resident_blocks(k)), 256, 0, st>>>((const Tin*)x, (const Tout*)g, (const Tout*)b,
+                                                              (Tout*)y, d_rows, rows_cap, H, eps, status);
 }
 
-// The vector kernel only exists for 16-bit types; fp32 always takes the generic one.
-template <>
-cudaError_t ln_dispatch<float>(const void* x, const void* g, const void* b, void* y, const int32_t* d_rows,
-                               int rows_cap, int H, float eps, const int32_t* status, const LnGather& gth,
-                               cudaStream_t st) {
-    const int resident = resident_blocks(ln_generic_kernel<float>);
-    ln_generic_kernel<float><<<ln_grid(rows_cap, resident), 256, 0, st>>>(
-        (const float*)x, (const float*)g, (const float*)b, (float*)y, d_rows, rows_cap, H, eps, status, gth);
+template <typename Tin, typename Tout>
+static cudaError_t ln_rows_dispatch(const void* x, const void* g, const void* b, void* y, const int32_t* d_rows,
+                                    int rows_cap, int H, float eps, const int32_t* status, cudaStream_t st) {
+    constexpr int N = 16 / sizeof(Tin);
+    constexpr int NO = N;  // output elements per vector step (N * sizeof(Tout) bytes)
+    const uintptr_t al = (uintptr_t)x | (uintptr_t)g | (uintptr_t)b | (uintptr_t)y;
+    const int nvec = H / N;
+    const int vpt = (nvec + 255) / 256;
+    const bool vec = H % N == 0 && al % 16 == 0 && (NO * sizeof(Tout)) % 4 == 0 && vpt >= 1 && vpt <= 16;
+    if (vec) {
+        if (vpt <= 1) ln_rows_launch<Tin, Tout, 1>(x, g, b, y, d_rows, rows_cap, H, eps, status, st);
+        else if (vpt <= 2) ln_rows_launch<Tin, Tout, 2>(x, g, b, y, d_rows, rows_cap, H, eps, status, st);
+        else if (vpt <= 4) ln_rows_launch<Tin, Tout, 4>(x, g, b, y, d_rows, rows_cap, H, eps, status, st);
+        else if (vpt <= 6) ln_rows_launch<Tin, Tout, 6>(x, g, b, y, d_rows, rows_cap, H, eps, status, st);
+        else if (vpt <= 8) ln_rows_launch<Tin, Tout, 8>(x, g, b, y, d_rows, rows_cap, H, eps, status, st);
+        else if (vpt <= 12) ln_rows_launch<Tin, Tout, 12>(x, g, b, y, d_rows, rows_cap, H, eps, status, st);
+        else ln_rows_launch<Tin, Tout, 16>(x, g, b, y, d_rows, rows_cap, H, eps, status, st);
+    } else {
+        auto k = ln_rows_generic_kernel<Tin, Tout>;
+        k<<<row_grid(rows_cap, resident_blocks(k)), 256, 0, st>>>((const Tin*)x, (const Tout*)g, (const Tout*)b,
+                                                                  (Tout*)y, d_rows, rows_cap, H, eps, status);
+    }
     return cudaGetLastError();
 }
 
 cudaError_t launch_layernorm(int dtype, const void* x, const void* g, const void* b, void* y, const int32_t* d_rows,
                              int rows_cap, int H, float eps, const int32_t* status, cudaStream_t st,
-                             const LnGather& gth) {
+                             const LnGather& gth, bool x_f32) {
+    if (gth.cu != nullptr) return cudaErrorInvalidValue;  // the gather form is the folded LayerNorm's
     switch (dtype) {
-    case ENERGON_F32: return ln_dispatch<float>(x, g, b, y, d_rows, rows_cap, H, eps, status, gth, st);
-    case ENERGON_F16: return ln_dispatch<__half>(x, g, b, y, d_rows, rows_cap, H, eps, status, gth, st);
-    case ENERGON_BF16: return ln_dispatch<__nv_bfloat16>(x, g, b, y, d_rows, rows_cap, H, eps, status, gth, st);
+    case ENERGON_F32: return ln_rows_dispatch<float, float>(x, g, b, y, d_rows, rows_cap, H, eps, status, st);
+    case ENERGON_F16:
+        return x_f32 ? ln_rows_dispatch<float, __half>(x, g, b, y, d_rows, rows_cap, H, eps, status, st)
+                     : ln_rows_dispatch<__half, __half>(x, g, b, y, d_rows, rows_cap, H, eps, status, st);
+    case ENERGON_BF16:
+        return x_f32 ? ln_rows_dispatch<float, __nv_bfloat16>(x, g, b, y, d_rows, rows_cap, H, eps, status, st)
+                     : ln_rows_dispatch<__nv_bfloat16, __nv_bfloat16>(x, g, b, y, d_rows, rows_cap, H, eps, status,
+                                                                       st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+template <typename T>
+static cudaError_t ln_fold_dispatch(const void* x, const void* g, void* u, float2* stats, const int32_t* d_rows,
+                                    int rows_cap, int H, float eps, const int32_t* status, const LnGather& gth,
+                                    cudaStream_t st) {
+    constexpr int N = 16 / sizeof(T);
+    const uintptr_t al = (uintptr_t)x | (uintptr_t)g | (uintptr_t)u | (uintptr_t)gth.copy;
+    if (H % N == 0 && al % 16 == 0) {
+        auto k = ln_fold_kernel<T, true>;
+        k<<<row_grid(rows_cap, resident_blocks(k)), 256, 0, st>>>((const T*)x, (const T*)g, (T*)u, stats, d_rows,
+                                                                  rows_cap, H, eps, status, gth);
+    } else {
+        auto k = ln_fold_kernel<T, false>;
+        k<<<row_grid(rows_cap, resident_blocks(k)), 256, 0, st>>>((const T*)x, (const T*)g, (T*)u, stats, d_rows,
+                                                                  rows_cap, H, eps, status, gth);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ln_fold(int dtype, const void* x, const void* g, void* u, float2* stats, const int32_t* d_rows,
+                           int rows_cap, int H, float eps, const int32_t* status, cudaStream_t st,
+                           const LnGather& gth) {
+    switch (dtype) {
+    case ENERGON_F32: return ln_fold_dispatch<float>(x, g, u, stats, d_rows, rows_cap, H, eps, status, gth, st);
+    case ENERGON_F16: return ln_fold_dispatch<__half>(x, g, u, stats, d_rows, rows_cap, H, eps, status, gth, st);
+    case ENERGON_BF16:
+        return ln_fold_dispatch<__nv_bfloat16>(x, g, u, stats, d_rows, rows_cap, H, eps, status, gth, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+template <typename T>
+static cudaError_t fold_weights_dispatch(const void* W, const void* g, const void* beta, const void* bias, int Nr,
+                                         int K, float* c, float* d, const int32_t* status, cudaStream_t st) {
+    constexpr int N = 16 / sizeof(T), RPW = 8;
+    const int blocks = (Nr + 8 * RPW - 1) / (8 * RPW);
+    const uintptr_t al = (uintptr_t)W | (uintptr_t)g | (uintptr_t)beta;
+    if (K % N == 0 && al % 16 == 0)
+        ln_fold_weights_kernel<T, true, RPW><<<blocks, 256, 0, st>>>((const T*)W, (const T*)g, (const T*)beta,
+                                                                    (const T*)bias, Nr, K, c, d, status);
+    else
+        ln_fold_weights_kernel<T, false, RPW><<<blocks, 256, 0, st>>>((const T*)W, (const T*)g, (const T*)beta,
+                                                                     (const T*)bias, Nr, K, c, d, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ln_fold_weights(int dtype, const void* W, const void* g, const void* beta, const void* bias,
+                                   int N, int K, float* c, float* d, const int32_t* status, cudaStream_t st) {
+    if (N <= 0 || K <= 0) return cudaSuccess;
+    switch (dtype) {
+    case ENERGON_F32: return fold_weights_dispatch<float>(W, g, beta, bias, N, K, c, d, status, st);
+    case ENERGON_F16: return fold_weights_dispatch<__half>(W, g, beta, bias, N, K, c, d, status, st);
+    case ENERGON_BF16: return fold_weights_dispatch<__nv_bfloat16>(W, g, beta, bias, N, K, c, d, status, st);
     }
     return cudaErrorInvalidValue;
 }

@@ -39,12 +39,17 @@ def layer_ws_offsets(H: int, F: int, batch: int, pad_len: int, elem: int) -> dic
     workspace (layout stated in include/energon_rce.h)."""
     R = align_up(batch * pad_len, 256)
     off, out = 0, {}
-    for name, cols in (("a", H), ("qkv", 3 * H), ("o", H), ("x1", H), ("f", F)):
+    for name, cols, eb in (("a", H, elem), ("qkv", 3 * H, elem), ("qk_lo", 2 * H if elem != 4 else 0, elem),
+                           ("o", H, elem), ("x1", H, 4), ("f", F, elem)):
         out[name] = (off, cols)
-        off = align_up(off + R * cols * elem, 1024)
+        off = align_up(off + R * cols * eb, 1024)
     p32 = 4 * 128 * max(3 * H, F) * 4 if batch * pad_len <= 128 else 0
     out["p32"] = (off, p32)
     off = align_up(off + p32, 1024)
+    out["stats"] = (off, 2)                       # float2 per row
+    off = align_up(off + R * 8, 1024)
+    out["fold"] = (off, 6 * H)                    # c [3H] then d [3H], fp32
+    off = align_up(off + 6 * H * 4, 1024)
     out["_layer_bytes"] = off
     return out
 
@@ -68,25 +73,22 @@ MAX_ABS = 2e-2   # stated max-abs bound for fp16/bf16 layer outputs
 REL_FRO = 5e-3   # stated relative Frobenius bound
 
 
-def check_end_to_end(g: np.ndarray, r: np.ndarray, dtype: int, label: str):
-    """End-to-end tolerance against the fp64 oracle.
-
-    rel-Frobenius <= 5e-3, as stated.  The max-abs bound of 2e-2 is applied above one
-    rounding unit of the storage type at the reference value and in scale-free form,
-    max |g - r| - ulp(r) <= 2e-2 * max(1, rms(r)): a 16-bit output cannot sit closer to an
-    fp64 value than its own rounding, and the roundings at every kernel boundary (inputs
-    of dot products over 12288 - 49152 terms) give errors proportional to the activation
-    scale, which reaches rms ~ 25 (|y| ~ 120) after 12 GPT-3 layers."""
+def check_end_to_end(g: np.ndarray, r: np.ndarray, dtype: int, label: str, max_abs: bool = True):
+    """Tolerance against the fp64 oracle for fp16 / bf16 layer outputs (fp32 accumulation):
+    relative Frobenius error <= 5e-3 and max-abs error <= 2e-2, the latter above one
+    rounding unit of the storage type at the reference value (a 16-bit output cannot sit
+    closer to an fp64 value than its own rounding): max |g - r| - ulp(r) <= 2e-2.
+    max_abs=False gates rel-Frobenius only (outputs of a stack of layers, where the stated
+    bound applies to each layer's output, not to their composition); the max-abs figures
+    are printed either way."""
     err = np.abs(g - r)
-    e_max, e_fro = float(err.max()), rel_frobenius(g, r)
-    rms = float(np.sqrt(np.mean(r ** 2))) if r.size else 0.0
+    e_max, e_fro = (float(err.max()) if err.size else 0.0), rel_frobenius(g, r)
     excess = float((err - ulp(r, dtype)).max()) if r.size else 0.0
-    bound = MAX_ABS * max(1.0, rms)
-    print(f"\n[{label}] max-abs {e_max:.3e} (beyond one ulp {excess:.3e}, bound {bound:.3e}, rms {rms:.2f}) "
-          f"rel-fro {e_fro:.3e}")
+    print(f"\n[{label}] max-abs {e_max:.3e} (beyond one ulp {excess:.3e}) rel-fro {e_fro:.3e}")
     assert e_fro <= REL_FRO, f"{label}: rel-Frobenius {e_fro:.3e} > {REL_FRO}"
-    assert excess <= bound, f"{label}: max-abs beyond one ulp {excess:.3e} > {bound:.3e}"
-    return e_max, e_fro
+    if max_abs:
+        assert excess <= MAX_ABS, f"{label}: max-abs beyond one ulp {excess:.3e} > {MAX_ABS}"
+    return e_max, e_fro, excess
 
 
 def rel_frobenius(g: np.ndarray, r: np.ndarray) -> float:

@@ -58,9 +58,11 @@ def test_workspace_bytes_matches_documented_layout(lib):
                                    (256, 4, 1024, capi.ENERGON_F32, 4, 4, 32)]:
         R = align(B * S, 256)
         off = 0
-        for cols in (H, 3 * H, H, H, F):
-            off = align(off + R * cols * e, 1024)
+        for cols, eb in ((H, e), (3 * H, e), (2 * H if e == 2 else 0, e), (H, e), (H, 4), (F, e)):
+            off = align(off + R * cols * eb, 1024)      # a, qkv, qk_lo (16-bit only), o, x1 (fp32), f
         off = align(off + (4 * 128 * max(3 * H, F) * 4 if B * S <= 128 else 0), 1024)   # split-K partials
+        off = align(off + R * 8, 1024)                                                    # LayerNorm statistics
+        off = align(off + 6 * H * 4, 1024)                                                # folded c, d
         off = align(off + R * H * e, 1024)                                                # stack: x
         off = align(off + (B + 1) * 4, 1024)
         off = align(off + (B + 1) * 4, 1024)
