@@ -511,7 +511,10 @@ def bench_stack(args, dist: Dist, wl, dev, stream, peaks: dict, want_cpu: bool, 
     res["roofline"] = gemm_roofline(H, T, e, g_launch, g_ms, peaks, traffic_from_profile())
     res["step_roofline"] = step_roofline(H, L, lengths, e, ms / args.steps, peaks)
     aux = {}
-    for name, nbytes in (("layernorm_remove", 3 * T * H * e), ("zero_pads", (B * S - T) * H * e)):
+    lo = 2 if e == 2 else 0   # the low halves of Q and K (16-bit types)
+    for name, nbytes in (("layernorm_remove", 3 * T * H * e), ("zero_pads", (B * S - T) * H * e),
+                         ("ln_fold", 2 * T * H * e + 8 * T), ("layernorm", T * H * (4 + e)),
+                         ("ln_fold_weights", 3 * H * H * e), ("attention", T * H * e * (3 + lo + 1))):
         if name in trace and trace[name][1] > 0:
             gbs = nbytes * trace[name][0] / (trace[name][1] / 1e3) / 1e9
             aux[name] = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",

@@ -216,43 +216,55 @@ __global__ void __launch_bounds__(256) ln_fold_kernel(const T* __restrict__ x, c
     }
 }
 
-// c[n] = sum_k g[k] W[n][k], d[n] = bias[n] + sum_k beta[k] W[n][k].  Each warp owns RPW
-// consecutive rows of W and walks K once, with g and beta loaded once per step for all
-// of its rows; lane-strided partial sums, then a fixed shuffle tree (deterministic).
-template <typename T, bool VEC, int RPW>
+// c[n] = sum_k g[k] W[n][k], d[n] = bias[n] + sum_k beta[k] W[n][k].  A block of 256
+// threads owns RPB consecutive rows of W; thread t takes the 16-byte vectors t, t + 256,
+// ... of every row, two vector steps at a time, so each thread has 2 * (RPB + 2) loads in
+// flight (the weights stream from HBM once).  Per-thread partial sums, then a fixed
+// shuffle tree and a fixed order across the warps (deterministic).
+template <typename T, bool VEC, int RPB>
 __global__ void __launch_bounds__(256) ln_fold_weights_kernel(const T* __restrict__ W, const T* __restrict__ g,
                                                               const T* __restrict__ beta, const T* __restrict__ bias,
                                                               int Nrows, int K, float* __restrict__ c,
                                                               float* __restrict__ d, const int32_t* status) {
     constexpr int N = VEC ? 16 / sizeof(T) : 1;
+    __shared__ float red[8][2 * RPB];
     if (status_bad(status)) return;
-    const int lane = threadIdx.x & 31;
-    const int n0 = (blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * RPW;
-    if (n0 >= Nrows) return;
-    float ac[RPW], ad[RPW];
-#pragma unroll
-    for (int i = 0; i < RPW; ++i) ac[i] = ad[i] = 0.0f;
+    const int n0 = blockIdx.x * RPB;
     const int nvec = K / N;
-    for (int idx = lane; idx < nvec; idx += 32) {
-        const int64_t e = (int64_t)idx * N;
-        float gv[N], bv[N];
-        load_f_ldg<T, N>(g + e, gv);
-        load_f_ldg<T, N>(beta + e, bv);
+    float ac[RPB], ad[RPB];
 #pragma unroll
-        for (int i = 0; i < RPW; ++i) {
-            if (n0 + i < Nrows) {
-                float wv[N];
-                load_f<T, N>(W + (int64_t)(n0 + i) * K + e, wv);
+    for (int i = 0; i < RPB; ++i) ac[i] = ad[i] = 0.0f;
+    for (int v0 = threadIdx.x; v0 < nvec; v0 += 2 * blockDim.x) {
+        // raw vectors first (all loads in flight), converted while accumulating
+        Pack<T, N> gp[2], bp[2], wp[2][RPB];
 #pragma unroll
-                for (int j = 0; j < N; ++j) {
-                    ac[i] = fmaf(gv[j], wv[j], ac[i]);
-                    ad[i] = fmaf(bv[j], wv[j], ad[i]);
+        for (int u = 0; u < 2; ++u) {
+            const int v = v0 + u * blockDim.x;
+            const int64_t e = (int64_t)(v < nvec ? v : 0) * N;
+            gp[u] = *reinterpret_cast<const Pack<T, N>*>(g + e);
+            bp[u] = *reinterpret_cast<const Pack<T, N>*>(beta + e);
+#pragma unroll
+            for (int i = 0; i < RPB; ++i)
+                wp[u][i] = *reinterpret_cast<const Pack<T, N>*>(W + (int64_t)(n0 + i < Nrows ? n0 + i : n0) * K + e);
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            if (v0 + u * (int)blockDim.x >= nvec) continue;
+#pragma unroll
+            for (int j = 0; j < N; ++j) {
+                const float gj = to_f(gp[u].v[j]), bj = to_f(bp[u].v[j]);
+#pragma unroll
+                for (int i = 0; i < RPB; ++i) {
+                    const float w = to_f(wp[u][i].v[j]);
+                    ac[i] = fmaf(gj, w, ac[i]);
+                    ad[i] = fmaf(bj, w, ad[i]);
                 }
             }
         }
     }
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
-    for (int i = 0; i < RPW; ++i) {
+    for (int i = 0; i < RPB; ++i) {
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
             ac[i] += __shfl_xor_sync(0xffffffffu, ac[i], o);
@@ -261,11 +273,17 @@ __global__ void __launch_bounds__(256) ln_fold_weights_kernel(const T* __restric
     }
     if (lane == 0) {
 #pragma unroll
-        for (int i = 0; i < RPW; ++i)
-            if (n0 + i < Nrows) {
-                c[n0 + i] = ac[i];
-                d[n0 + i] = ad[i] + (bias ? to_f(bias[n0 + i]) : 0.0f);
-            }
+        for (int i = 0; i < RPB; ++i) red[warp][i] = ac[i], red[warp][RPB + i] = ad[i];
+    }
+    __syncthreads();
+    if (threadIdx.x < 2 * RPB) {
+        float s = 0.0f;
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) s += red[w][threadIdx.x];
+        const int i = threadIdx.x % RPB;
+        if (n0 + i < Nrows) {
+            if (threadIdx.x < RPB) c[n0 + i] = s;
+            else d[n0 + i] = s + (bias ? to_f(bias[n0 + i]) : 0.0f);
+        }
     }
 }
 
@@ -372,14 +390,14 @@ cudaError_t launch_ln_fold(int dtype, const void* x, const void* g, void* u, flo
 template <typename T>
 static cudaError_t fold_weights_dispatch(const void* W, const void* g, const void* beta, const void* bias, int Nr,
                                          int K, float* c, float* d, const int32_t* status, cudaStream_t st) {
-    constexpr int N = 16 / sizeof(T), RPW = 8;
-    const int blocks = (Nr + 8 * RPW - 1) / (8 * RPW);
+    constexpr int N = 16 / sizeof(T), RPB = 8;
+    const int blocks = (Nr + RPB - 1) / RPB;
     const uintptr_t al = (uintptr_t)W | (uintptr_t)g | (uintptr_t)beta;
     if (K % N == 0 && al % 16 == 0)
-        ln_fold_weights_kernel<T, true, RPW><<<blocks, 256, 0, st>>>((const T*)W, (const T*)g, (const T*)beta,
+        ln_fold_weights_kernel<T, true, RPB><<<blocks, 256, 0, st>>>((const T*)W, (const T*)g, (const T*)beta,
                                                                     (const T*)bias, Nr, K, c, d, status);
     else
-        ln_fold_weights_kernel<T, false, RPW><<<blocks, 256, 0, st>>>((const T*)W, (const T*)g, (const T*)beta,
+        ln_fold_weights_kernel<T, false, RPB><<<blocks, 256, 0, st>>>((const T*)W, (const T*)g, (const T*)beta,
                                                                      (const T*)bias, Nr, K, c, d, status);
     return cudaGetLastError();
 }

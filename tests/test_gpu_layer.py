@@ -123,7 +123,7 @@ def layer_step_checks(res, shape, dtype, oracle_lib):
     if two_term:
         qkv[:, :2 * H] += it["qk_lo"]
     err = np.abs(qkv - (qkv_ref + shift))
-    tol = acc_tol(qkv_ref, H)
+    tol = np.full_like(qkv_ref, acc_tol(qkv_ref, H))
     tol[:, 2 * H:] += ulp(qkv_ref[:, 2 * H:], dtype)      # V: one rounding of the storage type
     if two_term:                                          # Q, K: the low half's own rounding
         tol[:, :2 * H] += ulp(it["qk_lo"], dtype) + 2.0 ** -22 * np.abs(qkv_ref[:, :2 * H])
