@@ -265,10 +265,10 @@ __device__ __forceinline__ void epilogue_store32(uint32_t* acc, const uint4* res
     }
 }
 
-// One warp drains 256 accumulator columns of its 32 TMEM lanes (= 32 output rows),
-// 32 columns at a time, row per thread; the TMEM load and the residual load of the next
-// chunk are issued before the current chunk is processed.
-template <typename T, int EPI>
+// One warp drains CH x 32 accumulator columns of its 32 TMEM lanes (= 32 output rows),
+// 32 columns at a time, row per thread; the TMEM load of the next chunk is issued before
+// the current chunk is processed.
+template <typename T, int EPI, int CH = 8>
 __device__ __forceinline__ void drain_256(uint32_t tbase, const TcParams& p, int row, int col_base, int M) {
     // The path for the one box per tile that holds row M - 1 (and boxes that straddle two
     // sequences when scattering): the residual is loaded chunk by chunk, not ahead.
@@ -281,13 +281,13 @@ __device__ __forceinline__ void drain_256(uint32_t tbase, const TcParams& p, int
     tmem_ld_x16(tbase, r[0]);
     tmem_ld_x16(tbase + 16, r[0] + 16);
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
+    for (int c = 0; c < CH; ++c) {
         const int cur = c & 1;
         const int col0 = col_base + c * 32;
         const bool live = row_ok && col0 < p.N;
         load_residual32<T, EPI>(p, row, col0, live, res);
         tmem_wait_ld_regs(r[cur]);
-        if (c + 1 < 8) {
+        if (c + 1 < CH) {
             tmem_ld_x16(tbase + (c + 1) * 32, r[cur ^ 1]);
             tmem_ld_x16(tbase + (c + 1) * 32 + 16, r[cur ^ 1] + 16);
         }
@@ -313,7 +313,7 @@ __device__ __forceinline__ uint32_t stage_off(int row, int chunk) {
 // `tempty_cluster`) as soon as its last columns are in registers.  Every row of the
 // warp must be valid (rows < M); the warp holding the last valid row takes drain_256
 // instead.  Returns false if a residual copy timed out.
-template <typename T, int EPI>
+template <typename T, int EPI, int CH = 8>
 __device__ __forceinline__ bool drain_256_staged(uint32_t tbase, const TcParams& p, const CUtensorMap* tmO,
                                                  const CUtensorMap* tmR, const CUtensorMap* tmL, uint8_t* sbuf,
                                                  uint64_t* rbar, uint32_t& rpar, int row_base, int out_row_base,
@@ -348,17 +348,17 @@ __device__ __forceinline__ bool drain_256_staged(uint32_t tbase, const TcParams&
         tmem_ld_x16(tbase + 16, r[0] + 16);
     }
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
+    for (int c = 0; c < CH; ++c) {
         const int cur = c & 1;
         const int rc = RB == 2 ? cur : 0;
         uint8_t* buf = sbuf + cur * 2048;
         if (RB == 1) {
             tmem_ld_x16(tbase + c * 32, r[0]);
             tmem_ld_x16(tbase + c * 32 + 16, r[0] + 16);
-            if (c + 1 < 8) load_residual32<T, EPI>(p, row, col_base + (c + 1) * 32, true, res[cur ^ 1]);
+            if (c + 1 < CH) load_residual32<T, EPI>(p, row, col_base + (c + 1) * 32, true, res[cur ^ 1]);
         }
         tmem_wait_ld_regs(r[rc]);
-        if (c + 1 < 8) {
+        if (c + 1 < CH) {
             if (RB == 2) {
                 tmem_ld_x16(tbase + (c + 1) * 32, r[rc ^ 1]);
                 tmem_ld_x16(tbase + (c + 1) * 32 + 16, r[rc ^ 1] + 16);
@@ -369,7 +369,7 @@ __device__ __forceinline__ bool drain_256_staged(uint32_t tbase, const TcParams&
             if (lane == 0) mbar_arrive_cluster(tempty_cluster);
         }
         const int col0 = col_base + c * 32;
-        if (TMA_RES && c + 1 < 8) {
+        if (TMA_RES && c + 1 < CH) {
             if (lane == 0) {
                 mbar_arrive_expect_tx(&rbar[cur ^ 1], 32 * 64);
                 tma_load_2d(sbuf + (cur ^ 1) * 2048, tmR, &rbar[cur ^ 1], col0 + 32, row_base);
@@ -439,6 +439,22 @@ __device__ __forceinline__ bool drain_256_staged(uint32_t tbase, const TcParams&
         }
     }
     return ok;
+}
+
+// Out-of-line forms of the two drains for the rare cases (the box holding row M - 1,
+// boxes that straddle two sequences, and the wave-tail units of half a tile's columns),
+// so that their registers do not add to the main path's.
+template <typename T, int EPI, int CH>
+__device__ __noinline__ void drain_rows_rare(uint32_t tbase, const TcParams& p, int row, int col_base, int M) {
+    drain_256<T, EPI, CH>(tbase, p, row, col_base, M);
+}
+template <typename T, int EPI, int CH>
+__device__ __noinline__ bool drain_staged_rare(uint32_t tbase, const TcParams& p, const CUtensorMap* tmO,
+                                               const CUtensorMap* tmR, const CUtensorMap* tmL, uint8_t* sbuf,
+                                               uint64_t* rbar, uint32_t& rpar, int row_base, int out_row_base,
+                                               int col_base, uint32_t tempty_cluster, const volatile int* abort_flag) {
+    return drain_256_staged<T, EPI, CH>(tbase, p, tmO, tmR, tmL, sbuf, rbar, rpar, row_base, out_row_base, col_base,
+                                        tempty_cluster, abort_flag);
 }
 
 // One warp writes its 32 rows x 256 accumulator columns as fp32 partial sums.
@@ -678,37 +694,44 @@ __device__ __forceinline__ void spin_ns(uint64_t ns) {
 // multicast to both CTAs (ring slots and accumulator hand-off); the peer's
 // epilogue hands accumulators back by arriving on the leader's barrier.
 //
-// MT = row tiles per pair tile.  MT = 1: 256 x 256 tiles, 6-stage ring of 32 KiB
-// per CTA, two 256-column TMEM accumulators so the epilogue of one tile overlaps
-// the MMAs of the next.  MT = 2: 512 x 256 tiles, the staged W panel feeds both
-// row tiles (a quarter less L2 -> SMEM traffic and shared-memory bandwidth per
-// flop), 4-stage ring of 48 KiB, one 512-column accumulator drained by eight
-// epilogue warps between tiles.
-template <int MT>
+// MT = row tiles per pair tile, BN = the tile's columns.  MT = 1: 256 x BN tiles,
+// 6-stage ring, two TMEM accumulators so the epilogue of one tile overlaps the MMAs of
+// the next.  MT = 2: 512 x BN tiles, the staged W panel feeds both row tiles (a quarter
+// less L2 -> SMEM traffic and shared-memory bandwidth per flop than MT = 1 at BN = 256),
+// 4-stage ring; the accumulators of two tiles fit in TMEM only for BN <= 128, otherwise
+// one accumulator is drained by eight epilogue warps between tiles.  BN in {128, 192, 256}:
+// narrower tiles leave less of the last round of tiles idle when N / BN tiles do not fill
+// the CTA pairs evenly.
+template <int MT, int BN = 256>
 struct PairCfg {
+    static_assert(BN % 64 == 0 && BN >= 128 && BN <= 256, "tile columns");
     static constexpr int STAGES = MT == 1 ? 6 : 4;
-    static constexpr int A_STAGE = MT * PA_STAGE;  // MT boxes of 128 rows x 64
-    static constexpr int STAGE = A_STAGE + PB_STAGE;
-    static constexpr int SLOTS = MT == 1 ? 2 : 1;  // TMEM accumulator slots
-    static constexpr int SLOT_COLS = MT * PBN;
+    static constexpr int A_STAGE = MT * PA_STAGE;        // MT boxes of 128 rows x 64
+    static constexpr int B_STAGE = (BN / 2) * PBK * 2;   // this CTA's BN / 2 rows of W x 64
+    static constexpr int STAGE = A_STAGE + B_STAGE;
+    static constexpr int SLOT_COLS = MT * BN;
+    static constexpr int SLOTS = 2 * SLOT_COLS <= 512 ? 2 : 1;  // TMEM accumulator slots
+    static constexpr int CH = BN / 32;                   // 32-column epilogue chunks per row tile
     static constexpr int EPI_WARPS = 4 * MT;
     static constexpr int THREADS = 128 + 32 * EPI_WARPS;
     static constexpr int EPI_STAGE = 4096;  // per epilogue warp: two 32 x 32 staging buffers
     static constexpr int SMEM = STAGES * STAGE + EPI_WARPS * EPI_STAGE + 1024 + 384;
+    static_assert(SMEM <= 232448, "shared memory per CTA");
 };
 
-template <typename T, int EPI, int MT>
-__global__ void __launch_bounds__(PairCfg<MT>::THREADS, 1)
+template <typename T, int EPI, int MT, int BN>
+__global__ void __launch_bounds__(PairCfg<MT, BN>::THREADS, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmR,
-                    const __grid_constant__ CUtensorMap tmL, const TcParams p) {
-    using C = PairCfg<MT>;
+                    const __grid_constant__ CUtensorMap tmBq, const __grid_constant__ CUtensorMap tmO,
+                    const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmL,
+                    const TcParams p) {
+    using C = PairCfg<MT, BN>;
     constexpr int NST = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = base;                    // [stage][MT][128 rows x 128 B]
-    uint8_t* sB = base + NST * C::A_STAGE;  // [stage][128 rows x 128 B]
-    uint8_t* sE = sB + NST * PB_STAGE;      // [epilogue warp][2][32 rows x 64 B]
+    uint8_t* sB = base + NST * C::A_STAGE;  // [stage][BN / 2 rows x 128 B]
+    uint8_t* sE = sB + NST * C::B_STAGE;    // [epilogue warp][2][32 rows x 64 B]
     uint64_t* full = reinterpret_cast<uint64_t*>(sE + C::EPI_WARPS * C::EPI_STAGE);
     uint64_t* empty = full + NST;
     uint64_t* tfull = empty + NST;
@@ -728,18 +751,29 @@ __global__ void __launch_bounds__(PairCfg<MT>::THREADS, 1)
     if (M <= 0) return;
     const int num_m = (M + PBM - 1) / PBM;               // 256-row tiles
     const int num_mt = (num_m + MT - 1) / MT;            // pair tiles along M
-    const int num_n = (p.N + PBN - 1) / PBN;
+    const int num_n = (p.N + BN - 1) / BN;
     const int total = num_mt * num_n;
-    // Wave tail: when the last round of pair tiles would leave more than half of the pairs
-    // idle, its tiles are issued as two half units of one row tile each, so the round takes
-    // half as long.  A row's arithmetic is the same in a half unit (the same MMA per row
-    // tile, the same K order), so results do not depend on how the tiles were cut.
-    int full_units = total, split_tiles = 0;
-    if (MT == 2 && total > npairs) {
+    // Wave tail: the tiles of the last, partly filled round are cut into s units (s = 1,
+    // 2 or 4, the one that finishes the round soonest): 2 = one row tile each, 4 = one row
+    // tile and half the columns each (MMA N = BN / 2).  A row's arithmetic is the same in
+    // every cut (the same MMA per row and column, the same K order), so results do not
+    // depend on how the tiles were cut.
+    int full_units = total, split_tiles = 0, split = 1;
+    if (MT == 2) {
         const int rem = total % npairs;
-        if (rem != 0 && 2 * rem <= npairs) full_units = total - rem, split_tiles = rem;
+        const int full_rounds = total / npairs;
+        if (rem != 0) {
+            // round time of the tail in units of a full tile: ceil(rem s / npairs) / s
+            int best = 1;
+            float best_t = (float)((rem + npairs - 1) / npairs);
+            for (int s = 2; s <= 4; s *= 2) {
+                const float t_s = (float)((rem * s + npairs - 1) / npairs) / (float)s;
+                if (t_s < best_t - 1e-6f) best_t = t_s, best = s;
+            }
+            if (best > 1) full_units = full_rounds * npairs, split_tiles = rem, split = best;
+        }
     }
-    const int units = full_units + 2 * split_tiles;
+    const int units = full_units + split * split_tiles;
     if (pair >= units) return;
     const int num_kb = (p.K + PBK - 1) / PBK;
     // Tile order: groups of 8 row tiles (2048 rows); inside a group every row tile of a
@@ -748,13 +782,19 @@ __global__ void __launch_bounds__(PairCfg<MT>::THREADS, 1)
     // on the four GPT-3 shapes it is within 1 % of every other order tried and ahead of
     // the rest; L2 eviction-priority hints made it 10 % slower.
     const int group = 8 / MT;
-    // unit u -> pair tile t and its row tiles [i0, i1)
-    auto unit_of = [&](int u, int& t, int& i0, int& i1) {
+    // unit u -> pair tile t, its row tiles [i0, i1) and column half h (-1: all columns)
+    auto unit_of = [&](int u, int& t, int& i0, int& i1, int& h) {
+        h = -1;
         if (u < full_units) {
             t = u, i0 = 0, i1 = MT;
         } else {
             const int v = u - full_units;
-            t = full_units + (v >> 1), i0 = v & 1, i1 = i0 + 1;
+            if (split == 2) {
+                t = full_units + (v >> 1), i0 = v & 1;
+            } else {
+                t = full_units + (v >> 2), i0 = (v >> 1) & 1, h = v & 1;
+            }
+            i1 = i0 + 1;
         }
     };
 
@@ -794,10 +834,10 @@ __global__ void __launch_bounds__(PairCfg<MT>::THREADS, 1)
         uint32_t phase = 0, pend_mask = 0, pend_par = 0;
         bool ok = true;
         for (int u = pair; u < units && ok; u += npairs) {
-            int t, i0, i1, mt, n;
-            unit_of(u, t, i0, i1);
+            int t, i0, i1, h, mt, n;
+            unit_of(u, t, i0, i1, h);
             tile_coords(t, num_mt, num_n, group, 0, mt, n);
-            const uint32_t tx = 2u * (uint32_t)((i1 - i0) * PA_STAGE + PB_STAGE);
+            const uint32_t tx = 2u * (uint32_t)((i1 - i0) * PA_STAGE + (h < 0 ? C::B_STAGE : C::B_STAGE / 2));
             for (int kb = 0; kb < num_kb; ++kb) {
                 if (!warp_wait<true>(&empty[stage], phase ^ 1u, abort_flag, p.timeout_ns)) {
                     ok = false;
@@ -811,7 +851,11 @@ __global__ void __launch_bounds__(PairCfg<MT>::THREADS, 1)
                         if (i >= i0 && i < i1)
                             tma_load_2d_pair(sA + stage * C::A_STAGE + i * PA_STAGE, &tmA, bar0, kb * PBK,
                                              (mt * MT + i) * PBM + (int)rank * 128);
-                    tma_load_2d_pair(sB + stage * PB_STAGE, &tmB, bar0, kb * PBK, n * PBN + (int)rank * 128);
+                    if (h < 0)
+                        tma_load_2d_pair(sB + stage * C::B_STAGE, &tmB, bar0, kb * PBK, n * BN + (int)rank * (BN / 2));
+                    else  // this CTA's BN / 4 rows of the column half
+                        tma_load_2d_pair(sB + stage * C::B_STAGE, &tmBq, bar0, kb * PBK,
+                                         n * BN + h * (BN / 2) + (int)rank * (BN / 4));
                 }
                 pend_mask |= 1u << stage;
                 pend_par = (pend_par & ~(1u << stage)) | (phase << stage);
@@ -836,13 +880,14 @@ __global__ void __launch_bounds__(PairCfg<MT>::THREADS, 1)
     } else if (warp == 1 && leader) {
         // ---------------------------------------------------------------- MMA issuer (leader CTA)
         constexpr uint32_t fmt = sizeof(T) == 2 && !std::is_same<T, __half>::value ? 1u : 0u;
-        constexpr uint32_t idesc = idesc_f16(fmt, PBM, PBN);
+        constexpr uint32_t idesc = idesc_f16(fmt, PBM, BN);
+        constexpr uint32_t idesc_h = idesc_f16(fmt, PBM, BN / 2);
         int stage = 0, local = 0;
         uint32_t phase = 0;
         bool ok = true;
         for (int u = pair; u < units && ok; u += npairs, ++local) {
-            int t, i0, i1;
-            unit_of(u, t, i0, i1);
+            int t, i0, i1, h;
+            unit_of(u, t, i0, i1, h);
             const int slot = local % C::SLOTS;
             const uint32_t use = (uint32_t)(local / C::SLOTS) & 1u;
             if (!warp_wait<true>(&tempty[slot], use ^ 1u, abort_flag, p.timeout_ns)) {
@@ -858,7 +903,7 @@ __global__ void __launch_bounds__(PairCfg<MT>::THREADS, 1)
                 }
                 tc_fence_after();
                 if (lane == 0) {
-                    const uint64_t b0 = smem_desc_k128(smem_u32(sB + stage * PB_STAGE));
+                    const uint64_t b0 = smem_desc_k128(smem_u32(sB + stage * C::B_STAGE));
                     // One thread issues an MMA every ~128 tensor cycles here, so the issue
                     // loops stay fully unrolled (a runtime-bounded loop measured 11 % slower).
                     if (i1 - i0 == MT) {
@@ -868,16 +913,22 @@ __global__ void __launch_bounds__(PairCfg<MT>::THREADS, 1)
                             for (int i = 0; i < MT; ++i) {
                                 const uint64_t a0 =
                                     smem_desc_k128(smem_u32(sA + stage * C::A_STAGE + i * PA_STAGE));
-                                umma_f16_pair(d_tmem + (uint32_t)(i * PBN), a0 + 2 * k, b0 + 2 * k, idesc,
+                                umma_f16_pair(d_tmem + (uint32_t)(i * BN), a0 + 2 * k, b0 + 2 * k, idesc,
                                               (kb | k) != 0 ? 1u : 0u);
                             }
                         }
-                    } else {
+                    } else if (h < 0) {
                         const uint64_t a0 = smem_desc_k128(smem_u32(sA + stage * C::A_STAGE + i0 * PA_STAGE));
-                        const uint32_t dt = d_tmem + (uint32_t)(i0 * PBN);
+                        const uint32_t dt = d_tmem + (uint32_t)(i0 * BN);
 #pragma unroll
                         for (int k = 0; k < PBK / 16; ++k)
                             umma_f16_pair(dt, a0 + 2 * k, b0 + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+                    } else {
+                        const uint64_t a0 = smem_desc_k128(smem_u32(sA + stage * C::A_STAGE + i0 * PA_STAGE));
+                        const uint32_t dt = d_tmem + (uint32_t)(i0 * BN + h * (BN / 2));
+#pragma unroll
+                        for (int k = 0; k < PBK / 16; ++k)
+                            umma_f16_pair(dt, a0 + 2 * k, b0 + 2 * k, idesc_h, (kb | k) != 0 ? 1u : 0u);
                     }
                     umma_commit_pair(&empty[stage], 0x3);
                 }
@@ -907,8 +958,8 @@ __global__ void __launch_bounds__(PairCfg<MT>::THREADS, 1)
         int local = 0;
         bool ok = true;
         for (int u = pair; u < units; u += npairs, ++local) {
-            int t, i0, i1;
-            unit_of(u, t, i0, i1);
+            int t, i0, i1, h;
+            unit_of(u, t, i0, i1, h);
             const int slot = local % C::SLOTS;
             const uint32_t use = (uint32_t)(local / C::SLOTS) & 1u;
             if (!warp_wait(&tfull[slot], use, abort_flag, p.timeout_ns)) {
@@ -922,8 +973,9 @@ __global__ void __launch_bounds__(PairCfg<MT>::THREADS, 1)
                 int mt, n;
                 tile_coords(t, num_mt, num_n, group, 0, mt, n);
                 const int row_base = (mt * MT + i) * PBM + (int)rank * 128 + q * 32;
+                const int cofs = h < 0 ? 0 : h * (BN / 2);  // first column of this unit in the tile
                 const uint32_t tbase =
-                    tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(slot * C::SLOT_COLS + i * PBN);
+                    tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(slot * C::SLOT_COLS + i * BN + cofs);
                 // a 32-row box is one TMA store when its rows are valid and (scattering)
                 // lie in one sequence, so that their padded rows are consecutive too
                 bool box = row_base + 32 <= M;
@@ -934,12 +986,18 @@ __global__ void __launch_bounds__(PairCfg<MT>::THREADS, 1)
                     box = row_base + 32 <= __ldg(p.scatter_cu + b + 1);
                     out_base = b * p.scatter_pad_len + (row_base - start);
                 }
-                if (box) {
-                    ok = drain_256_staged<T, EPI>(tbase, p, &tmO, &tmR, &tmL, sbuf, rb, rpar, row_base, out_base, n * PBN,
-                                                  tempty_cluster, abort_flag);
+                if (box && h < 0) {
+                    ok = drain_256_staged<T, EPI, C::CH>(tbase, p, &tmO, &tmR, &tmL, sbuf, rb, rpar, row_base,
+                                                         out_base, n * BN, tempty_cluster, abort_flag);
                     handed_back = ok;
+                } else if (box) {
+                    ok = drain_staged_rare<T, EPI, C::CH / 2>(tbase, p, &tmO, &tmR, &tmL, sbuf, rb, rpar, row_base,
+                                                              out_base, n * BN + cofs, tempty_cluster, abort_flag);
+                    handed_back = ok;
+                } else if (h < 0) {
+                    drain_rows_rare<T, EPI, C::CH>(tbase, p, row_base + lane, n * BN, M);
                 } else {
-                    drain_256<T, EPI>(tbase, p, row_base + lane, n * PBN, M);
+                    drain_rows_rare<T, EPI, C::CH / 2>(tbase, p, row_base + lane, n * BN + cofs, M);
                 }
             }
             if (!ok) break;
@@ -1046,17 +1104,17 @@ static cudaError_t tc_launch(const CUtensorMap& ta, const CUtensorMap& tb, const
     return cudaGetLastError();
 }
 
-template <typename T, int EPI, int MT>
-static cudaError_t tc2_launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to,
-                              const CUtensorMap& tr, const CUtensorMap& tl, const TcParams& p, int pairs,
-                              cudaStream_t st) {
-    using C = PairCfg<MT>;
+template <typename T, int EPI, int MT, int BN = 256>
+static cudaError_t tc2_launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tbq,
+                              const CUtensorMap& to, const CUtensorMap& tr, const CUtensorMap& tl, const TcParams& p,
+                              int pairs, cudaStream_t st) {
+    using C = PairCfg<MT, BN>;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    const void* kernel = (const void*)gemm_tc2_kernel<T, EPI, MT>;
+    const void* kernel = (const void*)gemm_tc2_kernel<T, EPI, MT, BN>;
     cudaError_t e = prepare_smem(kernel, C::SMEM);
     if (e != cudaSuccess) return e;
     // CTA pairs that fit on this device at once (the persistent grid)
@@ -1068,7 +1126,7 @@ static cudaError_t tc2_launch(const CUtensorMap& ta, const CUtensorMap& tb, cons
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int clusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&clusters, gemm_tc2_kernel<T, EPI, MT>, &cfg) != cudaSuccess ||
+        if (cudaOccupancyMaxActiveClusters(&clusters, gemm_tc2_kernel<T, EPI, MT, BN>, &cfg) != cudaSuccess ||
             clusters < 1)
             clusters = device_sm_count() / 2;
         (void)cudaGetLastError();
@@ -1082,18 +1140,18 @@ static cudaError_t tc2_launch(const CUtensorMap& ta, const CUtensorMap& tb, cons
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<T, EPI, MT>, ta, tb, to, tr, tl, p);
+    return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<T, EPI, MT, BN>, ta, tb, tbq, to, tr, tl, p);
 }
 
 template <typename T, int MT>
-static cudaError_t tc2_dispatch(int epi, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to,
-                                const CUtensorMap& tr, const CUtensorMap& tl, const TcParams& p, int pairs,
-                                cudaStream_t st) {
+static cudaError_t tc2_dispatch(int epi, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tbq,
+                                const CUtensorMap& to, const CUtensorMap& tr, const CUtensorMap& tl, const TcParams& p,
+                                int pairs, cudaStream_t st) {
     switch (epi) {
-    case EPI_LN_FOLD: return tc2_launch<T, EPI_LN_FOLD, MT>(ta, tb, to, tr, tl, p, pairs, st);
-    case EPI_BIAS_GELU: return tc2_launch<T, EPI_BIAS_GELU, MT>(ta, tb, to, tr, tl, p, pairs, st);
-    case EPI_RES_OUT32: return tc2_launch<T, EPI_RES_OUT32, MT>(ta, tb, to, tr, tl, p, pairs, st);
-    default: return tc2_launch<T, EPI_RES32, MT>(ta, tb, to, tr, tl, p, pairs, st);
+    case EPI_LN_FOLD: return tc2_launch<T, EPI_LN_FOLD, MT>(ta, tb, tbq, to, tr, tl, p, pairs, st);
+    case EPI_BIAS_GELU: return tc2_launch<T, EPI_BIAS_GELU, MT>(ta, tb, tbq, to, tr, tl, p, pairs, st);
+    case EPI_RES_OUT32: return tc2_launch<T, EPI_RES_OUT32, MT>(ta, tb, tbq, to, tr, tl, p, pairs, st);
+    default: return tc2_launch<T, EPI_RES32, MT>(ta, tb, tbq, to, tr, tl, p, pairs, st);
     }
 }
 
@@ -1182,6 +1240,13 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st, char* err, size_t
         }
         if (p.lo != nullptr) r5 = make_tmap_io(&tl, a.dtype, p.lo, p.lo_cols, a.M_cap);
         else tl = to;
+        // W boxes of half the height, for the wave-tail units that take half of a tile's columns
+        CUtensorMap tbq;
+        CUresult r6 = make_tmap(&tbq, a.dtype, a.W, a.K, a.N, 64);
+        if (r6 != CUDA_SUCCESS) {
+            if (err) snprintf(err, errlen, "cuTensorMapEncodeTiled failed (W half boxes: %d)", (int)r6);
+            return cudaErrorInvalidValue;
+        }
         if (r3 != CUDA_SUCCESS || r4 != CUDA_SUCCESS || r5 != CUDA_SUCCESS) {
             if (err)
                 snprintf(err, errlen, "cuTensorMapEncodeTiled failed (out: %d, residual: %d, low halves: %d)", (int)r3,
@@ -1189,10 +1254,10 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st, char* err, size_t
             return cudaErrorInvalidValue;
         }
         if (mt == 2)
-            return bf ? tc2_dispatch<__nv_bfloat16, 2>(a.epilogue, ta, tb, to, tr, tl, p, pairs, st)
-                      : tc2_dispatch<__half, 2>(a.epilogue, ta, tb, to, tr, tl, p, pairs, st);
-        return bf ? tc2_dispatch<__nv_bfloat16, 1>(a.epilogue, ta, tb, to, tr, tl, p, pairs, st)
-                  : tc2_dispatch<__half, 1>(a.epilogue, ta, tb, to, tr, tl, p, pairs, st);
+            return bf ? tc2_dispatch<__nv_bfloat16, 2>(a.epilogue, ta, tb, tbq, to, tr, tl, p, pairs, st)
+                      : tc2_dispatch<__half, 2>(a.epilogue, ta, tb, tbq, to, tr, tl, p, pairs, st);
+        return bf ? tc2_dispatch<__nv_bfloat16, 1>(a.epilogue, ta, tb, tbq, to, tr, tl, p, pairs, st)
+                  : tc2_dispatch<__half, 1>(a.epilogue, ta, tb, tbq, to, tr, tl, p, pairs, st);
     }
     const int num_m_cap = (a.M_cap + TBM - 1) / TBM, num_n = a.N / TBN;
     // Rows of A kept hot per raster group: about 48 MiB of the 126 MB L2.

@@ -122,13 +122,14 @@ def layer_step_checks(res, shape, dtype, oracle_lib):
     two_term = dtype != synth.F32
     if two_term:
         qkv[:, :2 * H] += it["qk_lo"]
-    err = np.abs(qkv - (qkv_ref + shift))
-    tol = np.full_like(qkv_ref, acc_tol(qkv_ref, H))
-    tol[:, 2 * H:] += ulp(qkv_ref[:, 2 * H:], dtype)      # V: one rounding of the storage type
+    want = qkv_ref + shift                                # the result on the GPU's own operand u
+    err = np.abs(qkv - want)
+    tol = np.full_like(want, acc_tol(want, H))
+    tol[:, 2 * H:] += ulp(want[:, 2 * H:], dtype)         # V: one rounding of the storage type
     if two_term:                                          # Q, K: the low half's own rounding
-        tol[:, :2 * H] += ulp(it["qk_lo"], dtype) + 2.0 ** -22 * np.abs(qkv_ref[:, :2 * H])
+        tol[:, :2 * H] += ulp(it["qk_lo"], dtype) + 2.0 ** -22 * np.abs(want[:, :2 * H])
     else:
-        tol += ulp(qkv_ref, dtype)
+        tol += ulp(want, dtype)
     report["qkv"] = float((err / tol).max()) if err.size else 0.0
     assert report["qkv"] <= 1.0, report
     # attention on the GPU's q, k (hi + lo) and v, one sequence at a time.  The tensor-core
@@ -257,15 +258,18 @@ def test_stack_packed_equals_padded_and_oracle(oracle_lib, dtype):
                              f"alone vs batch seq {b}")
 
 
-def test_gemm_wave_tail_cut_does_not_change_rows(oracle_lib):
-    """Hidden 1024, FFN 2560, 4096 valid tokens in a 16 x 512 batch.  On 148 SMs (74 CTA
-    pairs) the packed QKV and FFN1 GEMMs have 96 and 80 pair tiles, so their last round is
-    issued as half tiles; the padded run's 192 and 160 tiles are cut differently (not at
-    all, and 12 tiles).  Valid rows must agree bit for bit across the three modes, and
-    match the oracle."""
+@pytest.mark.parametrize("S,lens", [(512, [192, 320]), (256, [96, 160])])
+def test_gemm_wave_tail_cut_does_not_change_rows(oracle_lib, S, lens):
+    """Hidden 1024, FFN 2560, 16 sequences.  On 148 SMs (74 CTA pairs) the last, partly
+    filled round of 512 x 256 pair tiles is cut into half units (one row tile) or quarter
+    units (one row tile, 128 columns) depending on how many tiles it holds: with 4096
+    valid tokens the packed QKV and FFN1 GEMMs (96 and 80 tiles) cut their tail in halves;
+    with 2048 the out-projection and FFN2 (16 tiles) and FFN1 (40) cut it in quarters.
+    The padded runs (twice the rows) cut differently or not at all.  Valid rows must agree
+    bit for bit across the three modes, and match the oracle."""
     shape = synth.LayerShape(1024, 8, 2560)
-    B, S = 16, 512
-    lengths = np.array([192, 320] * 8, np.int32)
+    B = 16
+    lengths = np.array(lens * 8, np.int32)
     x = synth.normal((B, S, shape.hidden), 31, synth.TID_X, synth.F16)
     out1, st1, hw = stack_run(synth.F16, shape, 1, x, lengths, 31, NONZERO, 1)
     out0, st0, _ = stack_run(synth.F16, shape, 1, x, lengths, 31, NONZERO, 0)
