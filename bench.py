@@ -430,6 +430,23 @@ def upload_layers(wl, dist: Dist, dev, tdt, cpu: CpuSample | None = None):
     return dev_layers
 
 
+def prepare_folds(capi, cfg, dev_layers, H: int, dev, stream) -> float:
+    """The first LayerNorm's fold vectors of every layer, computed once (weight-load time);
+    returns their total device time in ms (CUDA events on the stream)."""
+    import torch
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    folds = [torch.empty(6 * H, dtype=torch.float32, device=dev) for _ in dev_layers]
+    torch.cuda.synchronize(dev)
+    a.record(stream)
+    for d, f in zip(dev_layers, folds):
+        capi.energon_layer_fold_weights(cfg, capi.make_weights(d), f, stream)
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    for d, f in zip(dev_layers, folds):
+        d["ln1_fold"] = f
+    return a.elapsed_time(b)
+
+
 def host_input(wl, tdt):
     import torch
     lengths, S = wl.lengths(), wl.padded_len()
@@ -467,10 +484,11 @@ def bench_stack(args, dist: Dist, wl, dev, stream, peaks: dict, want_cpu: bool, 
         x_np = x_host.numpy() if tdt != torch.bfloat16 else x_host.view(torch.int16).numpy().view(np.uint16)
         cpu = CpuSample(x_np, lengths, L, wl.shape.n_heads, budget_s=25.0, tokens=args.cpu_tokens)
     dev_layers = upload_layers(wl, dist, dev, tdt, cpu)
+    cfg = capi.make_config(H, wl.shape.n_heads, wl.shape.ffn, edt, wl.ln_eps)
+    fold_ms = prepare_folds(capi, cfg, dev_layers, H, dev, stream)
     tables = [capi.make_weights(d) for d in dev_layers]
     setup_s = time.perf_counter() - t0
 
-    cfg = capi.make_config(H, wl.shape.n_heads, wl.shape.ffn, edt, wl.ln_eps)
     ws_bytes = capi.energon_workspace_bytes(cfg, B, S)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
 
@@ -492,7 +510,11 @@ def bench_stack(args, dist: Dist, wl, dev, stream, peaks: dict, want_cpu: bool, 
     clk = clocks.stop()
     check_status("the timed steps")
     res = {"value": replica_value(dist.world, T, args.steps, ms), "ms_per_step": ms / args.steps,
-           "clocks": clk, "config": config_of(wl, S, T, dist.world), "setup_s": setup_s}
+           "clocks": clk, "config": config_of(wl, S, T, dist.world), "setup_s": setup_s,
+           "fold_vectors": {"prepared_at_weight_load": True, "ms_all_layers": fold_ms,
+                            "note": "c = W_qkv ln1_g and d = b_qkv + W_qkv ln1_b per layer "
+                                    "(energon_layer_fold_weights), computed once with the weights; "
+                                    "without them every step would recompute them (ms_all_layers)"}}
 
     # ---- a separate traced pass: per-kernel device time (one CUDA-event pair per launch)
     capi.energon_trace_start()
@@ -759,7 +781,8 @@ def run_energon(args, dist: Dist):
                 cw = synth.WORKLOADS[name]
                 c = bench_stack(cargs, dist, cw, dev, stream, peaks, False, full=False)
                 comp[name] = {k: c[k] for k in ("value", "ms_per_step", "config", "roofline", "step_roofline",
-                                                "padded_path", "kernels", "clocks", "setup_s") if k in c}
+                                                "padded_path", "kernels", "clocks", "setup_s", "fold_vectors")
+                              if k in c}
                 comp[name]["unit"] = UNIT
             comp["remove_rebuild"] = bench_packing(args, dist, synth.WORKLOADS["remove_rebuild"], dev, stream,
                                                    peaks, max(10, args.steps), args.warmup)
@@ -769,13 +792,31 @@ def run_energon(args, dist: Dist):
     dist.done()
 
 
+COST_SHAPES = ((8, 32), (16, 64), (32, 64), (32, 128), (64, 128), (64, 256))
+
+
+def cost_table(points, max_b: int, max_s: int):
+    """cost[b-1][s-1] of b sequences padded to s tokens: linear interpolation of the measured
+    (padded tokens, seconds) points in b * s, constant below the first point, extended along
+    the last segment above the last one."""
+    pts = sorted(points)
+    xs = np.array([p[0] for p in pts], np.float64)
+    ys = np.array([p[1] for p in pts], np.float64)
+    n = np.arange(1, max_b + 1)[:, None] * np.arange(1, max_s + 1)[None, :]
+    t = np.interp(n, xs, ys)
+    if len(xs) >= 2:
+        slope = (ys[-1] - ys[-2]) / (xs[-1] - xs[-2])
+        t = np.where(n > xs[-1], ys[-1] + slope * (n - xs[-1]), t)
+    return t.tolist()
+
+
 def run_batching(capi, synth, cfg, tables, L, tdt, dev, stream, tm: Timer, pool, st):
     """Serves 256 requests (lengths U[1, 256], all queued at once) in batches of at most 64:
     FIFO packing vs the dynamic-programming scheduler (energon_sched_plan), each batch padded
     to its longest request and run (a) on every padded row, as in the pages' comparison, and
     (b) with the padding eliminated.  The scheduler's cost table is this machine's: the
-    padded stack timed at four shapes (median of 3 after a warm-up run), least-squares fitted
-    as c0 + c1 * batch * padded length.  Every arm runs once to warm its batch shapes, then 3
+    padded stack timed at six shapes (median of 3 after a warm-up run), interpolated in the
+    padded token count (cost_table).  Every arm runs once to warm its batch shapes, then 3
     timed repeats (median, min, max).  Request activations are rows of the bench batch (the
     values do not change the work)."""
     import torch
@@ -800,21 +841,19 @@ def run_batching(capi, synth, cfg, tables, L, tdt, dev, stream, tm: Timer, pool,
                                            stream)
         return go
 
-    # machine costs of the padded stack
+    # machine costs of the padded stack, measured at six shapes; the cost of b sequences
+    # padded to s tokens is interpolated in the padded token count b * s (small batches are
+    # bound by streaming the weights, large ones by the GEMMs: not one straight line)
     pts = []
-    for b, s_len in ((max_b, max_s), (32, 128), (16, 64), (8, 32)):
+    for b, s_len in COST_SHAPES:
         x = torch.stack([pool[i % nb, :s_len] for i in range(b)]).contiguous()
         lens = torch.full((b,), s_len, dtype=torch.int32, device=dev)
         out = torch.empty_like(x)
         f = lambda: capi.energon_stack_forward(cfg, tables, L, x, lens, b, s_len, 0, out, st, ws, ws_bytes, stream)
         f()
         pts.append((b * s_len, statistics.median(tm.region(f, 1) for _ in range(reps)) / 1e3))
-    xs = np.array([p[0] for p in pts], np.float64)
-    ys = np.array([p[1] for p in pts], np.float64)
-    c1, c0 = np.polyfit(xs, ys, 1)
-    c1, c0 = max(float(c1), 1e-12), max(float(c0), 1e-6)
-    resid = float(np.sqrt(np.mean(((c0 + c1 * xs) - ys) ** 2 / ys ** 2)))
-    table = [[c0 + c1 * b * s_len for s_len in range(1, max_s + 1)] for b in range(1, max_b + 1)]
+    table = cost_table(pts, max_b, max_s)
+    lin = np.polyfit([p[0] for p in pts], [p[1] for p in pts], 1)
 
     fifo_of = capi.energon_sched_fifo(arrivals, max_b)
     fifo_groups = [[i for i in range(n_req) if fifo_of[i] == g] for g in range(max(fifo_of) + 1)]
@@ -823,9 +862,11 @@ def run_batching(capi, synth, cfg, tables, L, tdt, dev, stream, tm: Timer, pool,
     tokens = sum(lengths)
     res = {"requests": n_req, "max_batch": max_b, "valid_tokens": tokens,
            "lengths": "U[1, 256], seed 20260006, all queued at time 0",
-           "cost_model": {"c0_s": c0, "c1_s_per_padded_token": c1, "rms_rel_residual": resid,
-                          "fitted_on": "padded stack at 64x256, 32x128, 16x64, 8x32 (median of 3 each)",
-                          "points": [{"padded_tokens": int(a), "s": float(b)} for a, b in pts]}}
+           "cost_model": {"kind": "piecewise-linear in padded tokens between measured points",
+                          "measured_on": "padded stack at " + ", ".join(f"{b}x{s}" for b, s in COST_SHAPES)
+                                         + " (median of 3 each)",
+                          "points": [{"padded_tokens": int(a), "s": float(b)} for a, b in pts],
+                          "straight_line_fit": {"c0_s": float(lin[1]), "c1_s_per_padded_token": float(lin[0])}}}
     for name, groups in (("fifo", fifo_groups), ("dynamic", dyn_groups)):
         batches = [make_batch(g) for g in groups]
         padded_tokens = sum(b[0].shape[0] * b[3] for b in batches)

@@ -138,10 +138,17 @@ ENERGON_API int energon_rce_transpose_padding_remove(const void* heads, const in
 /* Weights of one pre-LN GPT decoder layer, all of the config's dtype, device:
  *   ln1_g, ln1_b [H]; w_qkv [3H, H], b_qkv [3H] (output columns Q | K | V, each
  *   head-major); w_o [H, H], b_o [H]; ln2_g, ln2_b [H]; w_1 [F, H], b_1 [F];
- *   w_2 [H, F], b_2 [H]. */
+ *   w_2 [H, F], b_2 [H].
+ *   ln1_fold: optional, fp32 [6H], 16-byte aligned: the first LayerNorm's fold
+ *   vectors c = W_qkv ln1_g [3H] followed by d = b_qkv + W_qkv ln1_b [3H], as
+ *   energon_layer_fold_weights writes them.  They depend on the weights only;
+ *   NULL makes every layer call compute them into its workspace (one pass over
+ *   W_qkv per call). */
 typedef struct {
     const void *ln1_g, *ln1_b, *w_qkv, *b_qkv, *w_o, *b_o, *ln2_g, *ln2_b, *w_1, *b_1, *w_2, *b_2;
+    const float* ln1_fold;
 } energon_layer_weights;
+
 
 /* hidden H, n_heads (head_dim = H / n_heads), ffn F, dtype (energon_dtype),
  * LayerNorm epsilon, gelu_tanh (1: tanh approximation as in GPT-2/3, 0: erf). */
@@ -150,6 +157,22 @@ typedef struct {
     float ln_eps;
     int gelu_tanh;
 } energon_layer_config;
+
+/*
+ * The first LayerNorm of a layer is folded into its QKV projection:
+ *   LN(x) W_qkv^T + b_qkv = rstd (x * ln1_g) W_qkv^T - mean rstd c + d
+ * with c = W_qkv ln1_g and d = b_qkv + W_qkv ln1_b, so that the tensor cores read
+ * the layer input itself (times ln1_g) rather than a rounded normalisation of it.
+ * This call computes c and d once for a set of weights (a weight-load step, like
+ * any layout preparation of the weights): fold [6H] fp32 device memory owned by
+ * the caller, 16-byte aligned; c, then d.  Reads w_qkv, b_qkv, ln1_g, ln1_b only.
+ * Asynchronous on `stream`; fp32 sums in a fixed order (the same values a layer
+ * call computes for itself when ln1_fold is NULL, bit for bit).
+ * Errors: invalid config, NULL pointer or misaligned fold -> ENERGON_ERR_* before
+ * any launch.
+ */
+ENERGON_API int energon_layer_fold_weights(const energon_layer_config* cfg, const energon_layer_weights* w,
+                                           float* fold, void* stream);
 
 /*
  * Workspace bytes that energon_layer_forward and energon_stack_forward need for

@@ -37,7 +37,8 @@ EXPORTED = ("energon_rce_offsets", "energon_rce_remove_padding", "energon_rce_re
             "energon_selftest_bounded_wait", "energon_set_wait_timeout_us", "energon_last_error",
             "energon_trace_start", "energon_trace_stop", "energon_rce_remove_padding_noalloc",
             "energon_rce_transpose_padding_rebuild", "energon_rce_transpose_padding_remove",
-            "energon_sched_plan", "energon_sched_fifo", "energon_kernel_binary_version")
+            "energon_sched_plan", "energon_sched_fifo", "energon_kernel_binary_version",
+            "energon_layer_fold_weights")
 ENERGON_NOALLOC_MAX_BATCH = 16384
 WEIGHT_FIELDS = ("ln1_g", "ln1_b", "w_qkv", "b_qkv", "w_o", "b_o",
                  "ln2_g", "ln2_b", "w_1", "b_1", "w_2", "b_2")
@@ -55,7 +56,7 @@ class energon_layer_config(ctypes.Structure):
 
 
 class energon_layer_weights(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_void_p) for n in WEIGHT_FIELDS]
+    _fields_ = [(n, ctypes.c_void_p) for n in WEIGHT_FIELDS] + [("ln1_fold", ctypes.c_void_p)]
 
 
 class energon_request(ctypes.Structure):
@@ -89,6 +90,7 @@ def load() -> ctypes.CDLL:
             "energon_stack_forward": ([cfgp, wp, ci, vp, vp, ci, ci, ci, vp, vp, vp, sz, vp], ci),
             "energon_selftest_bounded_wait": ([vp, u32, vp], ci),
             "energon_kernel_binary_version": ([ctypes.POINTER(ci)], ci),
+            "energon_layer_fold_weights": ([cfgp, wp, vp, vp], ci),
             "energon_set_wait_timeout_us": ([u32], None),
             "energon_last_error": ([], ctypes.c_char_p),
             "energon_trace_start": ([], ci),
@@ -216,6 +218,11 @@ def energon_selftest_bounded_wait(d_status, timeout_us, stream=None) -> None:
            "energon_selftest_bounded_wait")
 
 
+def energon_layer_fold_weights(cfg, weights, fold, stream=None) -> None:
+    _check(load().energon_layer_fold_weights(ctypes.byref(cfg), ctypes.byref(weights), _dev(fold, "fold"),
+                                             _stream(stream)), "energon_layer_fold_weights")
+
+
 def energon_kernel_binary_version() -> int:
     v = ctypes.c_int(0)
     _check(load().energon_kernel_binary_version(ctypes.byref(v)), "energon_kernel_binary_version")
@@ -281,5 +288,7 @@ def make_config(hidden: int, n_heads: int, ffn: int, dtype: int, ln_eps: float =
 
 
 def make_weights(tensors: dict) -> energon_layer_weights:
-    """Weight table of one layer from a dict of CUDA tensors (the dict must outlive its use)."""
-    return energon_layer_weights(*[_dev(tensors[n], n) for n in WEIGHT_FIELDS])
+    """Weight table of one layer from a dict of CUDA tensors (the dict must outlive its use);
+    an "ln1_fold" entry (fp32 [6H], from energon_layer_fold_weights) is optional."""
+    return energon_layer_weights(*[_dev(tensors[n], n) for n in WEIGHT_FIELDS],
+                                 _dev(tensors.get("ln1_fold"), "ln1_fold"))

@@ -184,6 +184,8 @@ int check_weights(const energon_layer_weights* w) {
                         w->ln2_g, w->ln2_b, w->w_1,   w->b_1,   w->w_2, w->b_2};
     for (const void* p : ps)
         if (!p) return fail(ENERGON_ERR_INVALID_ARGUMENT, "a weight pointer is NULL");
+    if ((uintptr_t)w->ln1_fold % 16 != 0)
+        return fail(ENERGON_ERR_MISALIGNED, "ln1_fold must be 16-byte aligned");
     return ENERGON_OK;
 }
 
@@ -241,16 +243,22 @@ int attention_sublayer(const energon_layer_config& c, const energon_layer_weight
                                         c.ln_eps, status, st, gth);
               }),
        padded ? "ln1 fold + remove" : "ln1 fold");
-    CK(traced("ln_fold_weights", st,
-              [&] {
-                  return launch_ln_fold_weights(c.dtype, w.w_qkv, w.ln1_g, w.ln1_b, w.b_qkv, 3 * H, H, ws.fold_c,
-                                                ws.fold_d, status, st);
-              }),
-       "ln1 fold weights");
+    // c and d: prepared with the weights (energon_layer_fold_weights), else computed here
+    const float* fold_c = w.ln1_fold;
+    const float* fold_d = w.ln1_fold ? w.ln1_fold + 3 * (size_t)H : nullptr;
+    if (fold_c == nullptr) {
+        CK(traced("ln_fold_weights", st,
+                  [&] {
+                      return launch_ln_fold_weights(c.dtype, w.w_qkv, w.ln1_g, w.ln1_b, w.b_qkv, 3 * H, H, ws.fold_c,
+                                                    ws.fold_d, status, st);
+                  }),
+           "ln1 fold weights");
+        fold_c = ws.fold_c, fold_d = ws.fold_d;
+    }
     GemmArgs g = gemm_base(c, cu, batch, max_len, status, ws);
     g.A = ws.a, g.W = w.w_qkv, g.bias = nullptr, g.residual = nullptr, g.out = ws.qkv;
     g.N = 3 * H, g.K = H, g.epilogue = EPI_LN_FOLD;
-    g.fold_stats = ws.stats, g.fold_c = ws.fold_c, g.fold_d = ws.fold_d;
+    g.fold_stats = ws.stats, g.fold_c = fold_c, g.fold_d = fold_d;
     g.lo = ws.qk_lo, g.lo_cols = ws.qk_lo ? 2 * H : 0;
     if (int r = run_gemm(g, st, "gemm_qkv")) return r;
     CK(traced("attention", st,
@@ -560,6 +568,20 @@ int energon_trace_stop(energon_trace_entry* entries, int capacity, int* n_entrie
     g_event_used = 0;
     if (n_entries) *n_entries = (int)agg.size();
     for (int i = 0; entries && i < capacity && i < (int)agg.size(); ++i) entries[i] = agg[i];
+    return ENERGON_OK;
+}
+
+int energon_layer_fold_weights(const energon_layer_config* cfg, const energon_layer_weights* w, float* fold,
+                               void* stream) {
+    g_last_error.clear();
+    if (int r = check_config(cfg)) return r;
+    if (!w || !w->w_qkv || !w->b_qkv || !w->ln1_g || !w->ln1_b || !fold)
+        return fail(ENERGON_ERR_INVALID_ARGUMENT, "fold weights: NULL pointer");
+    if ((uintptr_t)fold % 16 != 0) return fail(ENERGON_ERR_MISALIGNED, "fold weights: fold must be 16-byte aligned");
+    const int H = cfg->hidden;
+    CK(launch_ln_fold_weights(cfg->dtype, w->w_qkv, w->ln1_g, w->ln1_b, w->b_qkv, 3 * H, H, fold,
+                              fold + 3 * (size_t)H, nullptr, (cudaStream_t)stream),
+       "fold weights");
     return ENERGON_OK;
 }
 

@@ -9,7 +9,7 @@
 //    One thread block per row; each thread keeps its slice of the row in
 //    registers, so the row is read from HBM once and written once.
 //  - ln_fold_kernel: the LayerNorm before the QKV projection, folded into that
-//    GEMM.  It writes u = x * g (rounded to the storage type: exact when g is 1)
+//    GEMM (one warp per row; the row is streamed, not kept).  It writes u = x * g (rounded to the storage type: exact when g is 1)
 //    and the row statistics (rstd, mean * rstd); the GEMM's epilogue finishes
 //    LN(x) W^T + b = rstd (u W^T) - mean rstd c + d with c = W g, d = b + W beta
 //    (ln_fold_weights_kernel).  The tensor cores then see the layer input
@@ -175,18 +175,23 @@ __global__ void __launch_bounds__(256) ln_rows_generic_kernel(const Tin* __restr
 // ------------------------------------------------------------------ LayerNorm folded into the GEMM
 
 // u = x * g, stats = (rstd, mean * rstd); N elements per step (16-byte vectors when VEC).
+// One warp per row (the row is streamed, nothing of it is kept), eight rows per block:
+// every row of the batch is in flight at once, each lane with four vectors outstanding,
+// and the row statistics need only shuffles.
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(256) ln_fold_kernel(const T* __restrict__ x, const T* __restrict__ g,
                                                       T* __restrict__ u, float2* __restrict__ stats,
                                                       const int32_t* d_rows, int rows_cap, int H, float eps,
                                                       const int32_t* status, LnGather gth) {
     constexpr int N = VEC ? 16 / sizeof(T) : 1;
-    __shared__ float2 red[32];
+    constexpr int U = 4;
     if (status_bad(status)) return;
     const int rows = min(*d_rows, rows_cap);
     const int nvec = H / N;
+    const int lane = threadIdx.x & 31;
+    const int warps = gridDim.x * (blockDim.x >> 5);
     T* copy = static_cast<T*>(gth.copy);
-    for (int r = blockIdx.x; r < rows; r += gridDim.x) {
+    for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
         const int64_t src = ln_src_row(gth, r);
         if (src < 0) continue;
         const T* xr = x + src * H;
@@ -194,25 +199,41 @@ __global__ void __launch_bounds__(256) ln_fold_kernel(const T* __restrict__ x, c
         T* cr = copy ? copy + (int64_t)r * H : nullptr;
         const float x0 = to_f(xr[0]);
         float2 s = make_float2(0.0f, 0.0f);
-#pragma unroll 4
-        for (int idx = threadIdx.x; idx < nvec; idx += blockDim.x) {
-            const int64_t e = (int64_t)idx * N;
-            const Pack<T, N> xv = *reinterpret_cast<const Pack<T, N>*>(xr + e);
-            if (cr) *reinterpret_cast<Pack<T, N>*>(cr + e) = xv;
-            float gv[N], o[N];
-            load_f_ldg<T, N>(g + e, gv);
+        for (int base = lane; base < nvec; base += 32 * U) {
+            Pack<T, N> xv[U];
 #pragma unroll
-            for (int j = 0; j < N; ++j) {
-                const float v = to_f(xv.v[j]);
-                const float d = v - x0;
-                s.x += d;
-                s.y = fmaf(d, d, s.y);
-                o[j] = v * gv[j];
+            for (int k = 0; k < U; ++k) {
+                const int idx = base + 32 * k;
+                if (idx < nvec) xv[k] = *reinterpret_cast<const Pack<T, N>*>(xr + (int64_t)idx * N);
             }
-            store_f<T, N>(ur + e, o);
+#pragma unroll
+            for (int k = 0; k < U; ++k) {
+                const int idx = base + 32 * k;
+                if (idx >= nvec) continue;
+                const int64_t e = (int64_t)idx * N;
+                if (cr) *reinterpret_cast<Pack<T, N>*>(cr + e) = xv[k];
+                float gv[N], o[N];
+                load_f_ldg<T, N>(g + e, gv);
+#pragma unroll
+                for (int j = 0; j < N; ++j) {
+                    const float v = to_f(xv[k].v[j]);
+                    const float d = v - x0;
+                    s.x += d;
+                    s.y = fmaf(d, d, s.y);
+                    o[j] = v * gv[j];
+                }
+                store_f<T, N>(ur + e, o);
+            }
         }
-        const float2 mi = row_stats(x0, block_sum2(s, red), H, eps);
-        if (threadIdx.x == 0) stats[r] = make_float2(mi.y, mi.x * mi.y);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            s.x += __shfl_xor_sync(0xffffffffu, s.x, o);
+            s.y += __shfl_xor_sync(0xffffffffu, s.y, o);
+        }
+        if (lane == 0) {
+            const float2 mi = row_stats(x0, s, H, eps);
+            stats[r] = make_float2(mi.y, mi.x * mi.y);
+        }
     }
 }
 
@@ -363,14 +384,16 @@ static cudaError_t ln_fold_dispatch(const void* x, const void* g, void* u, float
                                     cudaStream_t st) {
     constexpr int N = 16 / sizeof(T);
     const uintptr_t al = (uintptr_t)x | (uintptr_t)g | (uintptr_t)u | (uintptr_t)gth.copy;
+    // eight rows (warps) per block, as many blocks as the rows need or the GPU holds
+    const int row_blocks = (rows_cap + 7) / 8;
     if (H % N == 0 && al % 16 == 0) {
         auto k = ln_fold_kernel<T, true>;
-        k<<<row_grid(rows_cap, resident_blocks(k)), 256, 0, st>>>((const T*)x, (const T*)g, (T*)u, stats, d_rows,
-                                                                  rows_cap, H, eps, status, gth);
+        k<<<row_grid(row_blocks, resident_blocks(k)), 256, 0, st>>>((const T*)x, (const T*)g, (T*)u, stats, d_rows,
+                                                                    rows_cap, H, eps, status, gth);
     } else {
         auto k = ln_fold_kernel<T, false>;
-        k<<<row_grid(rows_cap, resident_blocks(k)), 256, 0, st>>>((const T*)x, (const T*)g, (T*)u, stats, d_rows,
-                                                                  rows_cap, H, eps, status, gth);
+        k<<<row_grid(row_blocks, resident_blocks(k)), 256, 0, st>>>((const T*)x, (const T*)g, (T*)u, stats, d_rows,
+                                                                    rows_cap, H, eps, status, gth);
     }
     return cudaGetLastError();
 }

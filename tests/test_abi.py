@@ -143,7 +143,7 @@ def test_header_is_c_and_struct_layouts_match_the_binding(tmp_path):
     if shutil.which("gcc") is None:
         pytest.skip("gcc not available")
     structs = {
-        "energon_layer_weights": (capi.energon_layer_weights, list(capi.WEIGHT_FIELDS)),
+        "energon_layer_weights": (capi.energon_layer_weights, list(capi.WEIGHT_FIELDS) + ["ln1_fold"]),
         "energon_layer_config": (capi.energon_layer_config, ["hidden", "n_heads", "ffn", "dtype", "ln_eps",
                                                              "gelu_tanh"]),
         "energon_trace_entry": (capi.energon_trace_entry, ["name", "launches", "total_ms"]),

@@ -64,3 +64,16 @@ def test_fractions_of_burst_and_datasheet():
     assert r["frac_of_datasheet"] == pytest.approx(r["achieved"] / 2250.0)
     r = bench.gemm_roofline(12288, 32, 2, 40, 6.4, PEAKS, None)
     assert r["frac_of_datasheet"] == pytest.approx(r["achieved"] / 8000.0)
+
+
+def test_batching_cost_table_interpolates_the_measured_points():
+    pts = [(1024, 0.04), (256, 0.016), (4096, 0.15), (16384, 0.63)]
+    t = bench.cost_table(pts, 64, 256)
+    assert t[7][31] == pytest.approx(0.016)                 # 8 x 32 = 256 tokens: a measured point
+    assert t[0][0] == pytest.approx(0.016)                  # below the first point: its cost
+    assert t[31][127] == pytest.approx(0.15)                # 32 x 128 = 4096
+    assert t[15][159] == pytest.approx(0.04 + (2560 - 1024) / (4096 - 1024) * (0.15 - 0.04))   # 16 x 160
+    assert t[63][255] == pytest.approx(0.63)
+    # monotone in the padded token count, as the measured points are
+    flat = sorted(((b + 1) * (s + 1), t[b][s]) for b in range(64) for s in range(256))
+    assert all(flat[i][1] <= flat[i + 1][1] + 1e-15 for i in range(len(flat) - 1))

@@ -284,6 +284,46 @@ def test_gemm_wave_tail_cut_does_not_change_rows(oracle_lib, S, lens):
         check_end_to_end(to_f64(out1[b, :n]), ref[j, :n], synth.F16, f"wave-tail layer seq {b}")
 
 
+def test_prepared_fold_vectors_match_the_per_call_ones(oracle_lib):
+    """energon_layer_fold_weights writes c = W_qkv ln1_g and d = b_qkv + W_qkv ln1_b (checked
+    against the oracle's linear map); a stack given them returns, bit for bit, what it
+    returns when every layer computes them itself."""
+    shape = synth.LayerShape(256, 2, 1024)
+    H = shape.hidden
+    lengths = np.array([17, 64, 1, 0, 40, 64], np.int32)
+    B, S, L = len(lengths), 64, 2
+    x = synth.normal((B, S, H), 12, synth.TID_X, synth.F16)
+    out_call, st1, hw = stack_run(synth.F16, shape, L, x, lengths, 12, NONZERO, 1)
+    cfg = capi.make_config(H, shape.n_heads, shape.ffn, capi.ENERGON_F16)
+    keep = [gpu_layer_weights(shape, l, 12, synth.F16, NONZERO) for l in range(L)]
+    for host, dev in keep:
+        fold = torch.full((6 * H,), float("nan"), dtype=torch.float32, device="cuda")
+        capi.energon_layer_fold_weights(cfg, capi.make_weights(dev), fold)
+        dev["ln1_fold"] = fold
+        torch.cuda.synchronize()
+        g = synth.to_f64(host["ln1_g"], synth.F16)[None, :]
+        beta = synth.to_f64(host["ln1_b"], synth.F16)[None, :]
+        c_ref = oracle_lib.linear(g, host["w_qkv"])[0]
+        d_ref = oracle_lib.linear(beta, host["w_qkv"], host["b_qkv"])[0]
+        got = fold.double().cpu().numpy()
+        scale = 8 * np.sqrt(H) * 2.0 ** -24
+        assert np.abs(got[:3 * H] - c_ref).max() <= scale * np.abs(c_ref).max() + 1e-30
+        assert np.abs(got[3 * H:] - d_ref).max() <= scale * np.abs(d_ref).max() + 1e-30
+    ws_bytes = capi.energon_workspace_bytes(cfg, B, S)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    d_in = to_device(x, synth.F16)
+    out_prep = torch.empty_like(d_in)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tables = [capi.make_weights(d) for _, d in keep]
+    capi.energon_trace_start()
+    capi.energon_stack_forward(cfg, tables, L, d_in, torch.from_numpy(lengths).cuda(), B, S, 1, out_prep, st, ws,
+                               ws_bytes)
+    trace = capi.energon_trace_stop()
+    assert st1 == 0 and int(st.item()) == 0
+    assert "ln_fold_weights" not in trace                 # nothing recomputed per call
+    assert torch.equal(out_prep.view(torch.int16), out_call.view(torch.int16))
+
+
 def test_stack_invalid_lengths_and_empty_batch():
     shape = synth.LayerShape(256, 2, 512)
     x = synth.normal((3, 16, 256), 4, synth.TID_X, synth.F16)
