@@ -241,17 +241,26 @@ def reference_layers(args, oracle, wl, lengths, x):
 # ----------------------------------------------------------------------------- our arm
 
 
+def gemm_device_code_hash() -> str:
+    """sha256 (16 hex digits) of the GEMM's device code: gemm_tc.cu up to its host-side
+    section, plus the shared device helpers.  Host-side changes leave it unchanged."""
+    csrc = os.path.join(ROOT, "padding_free_varlen_b200", "csrc")
+    src = open(os.path.join(csrc, "gemm_tc.cu")).read()
+    cut = src.find("// ------------------------------------------------------------------ host side")
+    h = hashlib.sha256((src[:cut] if cut >= 0 else src).encode())
+    h.update(open(os.path.join(csrc, "common.cuh"), "rb").read())
+    return h.hexdigest()[:16]
+
+
 def traffic_from_profile() -> int | None:
-    """DRAM bytes per launch of the GEMM kernel from the committed ncu summary, if the kernel
-    source has not changed since the counters were taken."""
+    """DRAM bytes per launch of the GEMM kernel from the committed ncu summary, if the GEMM's
+    device code has not changed since the counters were taken."""
     path = os.path.join(ROOT, "profiles", "gemm_tc_traffic.json")
-    src = os.path.join(ROOT, "padding_free_varlen_b200", "csrc", "gemm_tc.cu")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         d = json.load(f)
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    if d.get("source_sha256_16") != h:
+    if d.get("device_code_sha256_16") != gemm_device_code_hash():
         return None
     return d.get("dram_bytes_per_launch_scaled")
 
