@@ -7,21 +7,26 @@
 // head j and position s:  o_j(s) = sum_{t <= s} softmax_t(q_j(s) . k_j(t) / sqrt(d)) v_j(t).
 //
 // One CTA = 128 queries of one (sequence, head), head_dim 128, 128 threads;
-// thread i owns query row i, which is TMEM lane i.  Per block of KB keys:
+// thread i owns query row i, which is TMEM lane i.  Per block of 64 keys:
 //   TMA   Q (once) and the key block's K and V tiles straight from the packed
 //         qkv rows (128-byte swizzle), plus the low halves of Q and K (qk_lo)
-//   MMA   S = Q K^T (tcgen05.mma kind::f16, M = 128, N = KB, K = 128) into TMEM
-//         columns 0..KB-1, from the two-term Q and K: Qh Kh^T + Qh Kl^T + Ql Kh^T
+//   MMA   S = Q K^T (tcgen05.mma kind::f16, M = 128, N = 64, K = 128) into TMEM
+//         columns 0..63, from the two-term Q and K: Qh Kh^T + Qh Kl^T + Ql Kh^T
 //   ALU   each thread reads its S row from TMEM, applies the causal mask, keeps
 //         a running max / sum (online softmax, fp32, exp2 with the scale folded
-//         in) and writes P, rounded to the storage type, into shared memory
-//   MMA   O += P V  (V used as an MN-major operand, no transpose) into TMEM 128..255
-// With the low halves, KB = 64 keeps a CTA at 112 KiB of shared memory and 256
-// TMEM columns, so that two CTAs share an SM and one's copies and MMAs overlap
-// the other's softmax.  Keys past the sequence are masked; their V rows are
-// zeroed in shared memory first, so stale workspace contents can never reach a
-// valid row (0 * NaN).  A query tile visits the key blocks 0 .. its diagonal that
-// hold keys of the sequence, whether the sequence is packed or padded.
+//         in) and writes P, rounded to the storage type, back into TMEM
+//         (columns 64..95, two keys per column)
+//   MMA   O += P V with P read from TMEM and V from shared memory as an MN-major
+//         operand (no transpose), into TMEM columns 128..255
+// P never touches shared memory, so the K buffer is free as soon as the S MMAs
+// are done: the next block's K is fetched while this block's softmax runs, and
+// the next block's V while the next S and softmax run.  A CTA holds 112 KiB of
+// shared memory and 256 TMEM columns, so that two CTAs share an SM and one's
+// copies and MMAs overlap the other's softmax.  Keys past the sequence are
+// masked; their V rows are zeroed in shared memory first, so stale workspace
+// contents can never reach a valid row (0 * NaN).  A query tile visits the key
+// blocks 0 .. its diagonal that hold keys of the sequence, whether the sequence
+// is packed or padded.
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -35,19 +40,41 @@ namespace energon {
 namespace {
 constexpr int ATQ = 128;                 // queries per CTA
 constexpr int AHD = 128;                 // head dim
+constexpr int KB = 64;                   // keys per block
 constexpr int QTILE = 128 * 64 * 2;      // 128 rows x 64 columns of 16-bit = 16 KiB, one swizzle block column
-constexpr uint32_t AT_TMEM_COLS = 256;   // S: 0..KB-1, O: 128..255
-constexpr int KB_LO = 64;                // key block with the low halves (two CTAs per SM)
+constexpr int KTILE = KB * 64 * 2;       // KB rows x 64 columns of 16-bit
+constexpr uint32_t AT_TMEM_COLS = 256;   // S: 0..63, P: 64..95, O: 128..255
+constexpr uint32_t P_COL = 64, O_COL = 128;
 
-// Shared memory of one CTA: Q (2 tiles), the key block's K and V (2 boxes each of KB rows
-// x 64 columns), with LO the low halves of Q (2 tiles) and K (2 boxes); 128 bytes of
-// barriers; slack to align the tiles to 1024 bytes.
-template <int KB, bool LO>
+// Shared memory of one CTA: Q (2 tiles), the key block's K and V (2 boxes each of 64 rows
+// x 64 columns), with LO the low halves of Q (2 tiles) and K (2 boxes); barriers in the
+// alignment slack or after the tiles.
+template <bool LO>
 struct AttnCfg {
-    static constexpr int KTILE = KB * 64 * 2;
     static constexpr int TILES = (LO ? 4 : 2) * QTILE + (LO ? 6 : 4) * KTILE;
-    static constexpr int SMEM = TILES + 1024;  // barriers go in the alignment slack or after the tiles
+    static constexpr int SMEM = TILES + 1024;
 };
+
+// O (or S) += A B with A (M = 128 rows, 16-bit, two per 32-bit column) read from TMEM.
+__device__ __forceinline__ void umma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                                uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// 32 lanes x 32 bits, 16 consecutive columns per thread.
+__device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t* r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
 }  // namespace
 
 struct AttnTcParams {
@@ -67,29 +94,31 @@ __device__ __forceinline__ bool block_wait(uint64_t* bar, uint32_t parity, uint6
 }
 
 // tmq / tmql: Q and its low halves in boxes of 128 rows; tmk / tmkl: K, V and K's low
-// halves in boxes of KB rows.
-template <typename T, int KB, bool LO>
+// halves in boxes of 64 rows.
+template <typename T, bool LO>
 __global__ void __launch_bounds__(128) attn_tc_kernel(const __grid_constant__ CUtensorMap tmq,
                                                       const __grid_constant__ CUtensorMap tmk,
                                                       const __grid_constant__ CUtensorMap tmql,
                                                       const __grid_constant__ CUtensorMap tmkl, const AttnTcParams p) {
-    using C = AttnCfg<KB, LO>;
-    constexpr int KT = C::KTILE;
+    using C = AttnCfg<LO>;
+    constexpr int KT = KTILE;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* sQ = base;                    // Q: head dims 0..63 | 64..127
-    uint8_t* sQl = sQ + 2 * QTILE;         // low half of Q (LO)
-    uint8_t* sK = sQ + (LO ? 4 : 2) * QTILE;  // K: head dims 0..63 | 64..127; then P (128 x KB)
-    uint8_t* sKl = sK + 2 * KT;            // low half of K (LO)
-    uint8_t* sV = sK + (LO ? 4 : 2) * KT;  // V: head dims 0..63 | 64..127, one row per key
+    uint8_t* sQ = base;                       // Q: head dims 0..63 | 64..127
+    uint8_t* sQl = sQ + 2 * QTILE;            // low half of Q (LO)
+    uint8_t* sK = sQ + (LO ? 4 : 2) * QTILE;  // K: head dims 0..63 | 64..127
+    uint8_t* sKl = sK + 2 * KT;               // low half of K (LO)
+    uint8_t* sV = sK + (LO ? 4 : 2) * KT;     // V: head dims 0..63 | 64..127, one row per key
     // barriers: in the alignment slack when it holds them, else after the tiles
     uint64_t* bars = (base - smem_raw >= 128) ? reinterpret_cast<uint64_t*>(smem_raw)
                                               : reinterpret_cast<uint64_t*>(base + C::TILES);
-    uint64_t* bar_q = bars;
-    uint64_t* bar_kv = bars + 1;
-    uint64_t* bar_mma = bars + 2;
-    uint64_t* drain = bars + 3;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
+    uint64_t* bar_q = bars;      // Q landed
+    uint64_t* bar_k = bars + 1;  // the block's K landed
+    uint64_t* bar_v = bars + 2;  // the block's V landed
+    uint64_t* bar_s = bars + 3;  // the S MMAs (and every MMA before them) done
+    uint64_t* bar_o = bars + 4;  // the PV MMAs done
+    uint64_t* drain = bars + 5;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 6);
 
     const int tid = threadIdx.x, warp = tid >> 5;
     if (status_bad(p.status)) return;
@@ -102,7 +131,7 @@ __global__ void __launch_bounds__(128) attn_tc_kernel(const __grid_constant__ CU
     const bool row_ok = q < len;
 
     if (tid == 0) {
-        for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < 6; ++i) mbar_init(&bars[i], 1);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -114,24 +143,29 @@ __global__ void __launch_bounds__(128) attn_tc_kernel(const __grid_constant__ CU
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const uint32_t S_t = tmem + lane_base, O_t = tmem + lane_base + 128;
+    const uint32_t S_t = tmem + lane_base, P_t = tmem + lane_base + P_COL, O_t = tmem + lane_base + O_COL;
 
     // Q | K | V at columns j*d, H + j*d, 2H + j*d of qkv; the low halves at j*d, H + j*d of qk_lo
     const int colQ = j * AHD, colK = p.H + j * AHD, colV = 2 * p.H + j * AHD;
-    bool q_pending = false, kv_pending = false;
-    uint32_t kv_parity = 0;
-    auto issue_kv = [&](int kb) {
+    bool q_pending = false, k_pending = false, v_pending = false;  // thread 0's copies in flight
+    uint32_t k_par = 0, v_par = 0;
+    auto issue_k = [&](int kb) {
         const int y = start + kb * KB;
-        mbar_arrive_expect_tx(bar_kv, (LO ? 6 : 4) * KT);
-        tma_load_2d(sK, &tmk, bar_kv, colK, y);
-        tma_load_2d(sK + KT, &tmk, bar_kv, colK + 64, y);
-        tma_load_2d(sV, &tmk, bar_kv, colV, y);
-        tma_load_2d(sV + KT, &tmk, bar_kv, colV + 64, y);
+        mbar_arrive_expect_tx(bar_k, (LO ? 4 : 2) * KT);
+        tma_load_2d(sK, &tmk, bar_k, colK, y);
+        tma_load_2d(sK + KT, &tmk, bar_k, colK + 64, y);
         if (LO) {
-            tma_load_2d(sKl, &tmkl, bar_kv, colK, y);
-            tma_load_2d(sKl + KT, &tmkl, bar_kv, colK + 64, y);
+            tma_load_2d(sKl, &tmkl, bar_k, colK, y);
+            tma_load_2d(sKl + KT, &tmkl, bar_k, colK + 64, y);
         }
-        kv_pending = true;
+        k_pending = true;
+    };
+    auto issue_v = [&](int kb) {
+        const int y = start + kb * KB;
+        mbar_arrive_expect_tx(bar_v, 2 * KT);
+        tma_load_2d(sV, &tmk, bar_v, colV, y);
+        tma_load_2d(sV + KT, &tmk, bar_v, colV + 64, y);
+        v_pending = true;
     };
     if (tid == 0) {
         tma_prefetch_desc(&tmq);
@@ -148,34 +182,23 @@ __global__ void __launch_bounds__(128) attn_tc_kernel(const __grid_constant__ CU
             tma_load_2d(sQl + QTILE, &tmql, bar_q, colQ + 64, start + q0);
         }
         q_pending = true;
-        issue_kv(0);
+        issue_k(0);
+        issue_v(0);
     }
     constexpr uint32_t fmt = std::is_same<T, __half>::value ? 0u : 1u;
     constexpr uint32_t idesc_s = idesc_f16(fmt, ATQ, KB, 0);
     constexpr uint32_t idesc_o = idesc_f16(fmt, ATQ, AHD, 1);
 
     float m_i = -INFINITY, l_i = 0.0f;
-    uint32_t mma_phase = 0;
+    uint32_t s_phase = 0, o_phase = 0;
     bool ok = block_wait(bar_q, 0, p.timeout_ns);
     if (ok) q_pending = false;
     uint32_t r[32];
     for (int kb = 0; ok && kb < n_kb; ++kb) {
-        ok = block_wait(bar_kv, kv_parity, p.timeout_ns);
+        ok = block_wait(bar_k, k_par, p.timeout_ns);
         if (!ok) break;
-        kv_pending = false;
-        kv_parity ^= 1u;
-        const int kbase = kb * KB;
-        if (tid < KB && kbase + tid >= len) {  // key row past the sequence: zero its V row
-            const uint4 z = make_uint4(0, 0, 0, 0);
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                reinterpret_cast<uint4*>(sV + tid * 128)[c] = z;
-                reinterpret_cast<uint4*>(sV + KT + tid * 128)[c] = z;
-            }
-            fence_proxy_async_smem();
-        }
-        tc_fence_before();
-        __syncthreads();
+        k_pending = false;
+        k_par ^= 1u;
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
@@ -190,14 +213,18 @@ __global__ void __launch_bounds__(128) attn_tc_kernel(const __grid_constant__ CU
                     umma_f16(tmem, al, bk, idesc_s, 1u);
                 }
             }
-            umma_commit(bar_mma);
+            umma_commit(bar_s);
         }
-        ok = block_wait(bar_mma, mma_phase, p.timeout_ns);
-        mma_phase ^= 1u;
+        ok = block_wait(bar_s, s_phase, p.timeout_ns);
+        s_phase ^= 1u;
         if (!ok) break;
         tc_fence_after();
+        // The S MMAs are done, and every MMA before them (the previous block's PV): the K
+        // buffer is free for the next block, O holds the sum over the earlier blocks.
+        if (tid == 0 && kb + 1 < n_kb) issue_k(kb + 1);
 
         // ---- online softmax of this thread's row
+        const int kbase = kb * KB;
         const int nvalid = row_ok ? min(KB, q - kbase + 1) : 0;  // keys kbase .. kbase+nvalid-1 are visible
         float mx = -INFINITY;
 #pragma unroll 1
@@ -211,28 +238,22 @@ __global__ void __launch_bounds__(128) attn_tc_kernel(const __grid_constant__ CU
         const float m_new = row_ok ? fmaxf(m_i, mx) : 0.0f;
         const float alpha = row_ok ? exp2f((m_i - m_new) * p.scale_log2e) : 1.0f;
         float rs = 0.0f;
-        uint8_t* sP = sK;  // P: 128 rows x KB keys, 128-byte rows, one swizzle block column per 64 keys
 #pragma unroll 1
         for (int c = 0; c < KB / 32; ++c) {
             tmem_ld_x32(S_t + c * 32, r);
             tmem_wait_ld();
-            float pv[32];
+            uint32_t pk[16];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                pv[e] = (c * 32 + e < nvalid) ? exp2f((__uint_as_float(r[e]) - m_new) * p.scale_log2e) : 0.0f;
-                rs += pv[e];
+            for (int e = 0; e < 16; ++e) {
+                const float p0 = (c * 32 + 2 * e < nvalid)
+                                     ? exp2f((__uint_as_float(r[2 * e]) - m_new) * p.scale_log2e) : 0.0f;
+                const float p1 = (c * 32 + 2 * e + 1 < nvalid)
+                                     ? exp2f((__uint_as_float(r[2 * e + 1]) - m_new) * p.scale_log2e) : 0.0f;
+                rs += p0;
+                rs += p1;
+                pk[e] = pack2<T>(p0, p1);  // keys 2e, 2e + 1 of this chunk in one column
             }
-            // keys c*32 .. c*32+31: swizzle block c/2, 16-byte chunks (c%2)*4 .. +3 of row tid
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {
-                uint4 w;
-                w.x = pack2<T>(pv[8 * g + 0], pv[8 * g + 1]);
-                w.y = pack2<T>(pv[8 * g + 2], pv[8 * g + 3]);
-                w.z = pack2<T>(pv[8 * g + 4], pv[8 * g + 5]);
-                w.w = pack2<T>(pv[8 * g + 6], pv[8 * g + 7]);
-                const int ch = (c & 1) * 4 + g;
-                *reinterpret_cast<uint4*>(sP + (c >> 1) * QTILE + tid * 128 + ((ch ^ (tid & 7)) << 4)) = w;
-            }
+            tmem_st_x16(P_t + c * 16, pk);
         }
         l_i = l_i * alpha + rs;
         if (row_ok) m_i = m_new;
@@ -245,26 +266,38 @@ __global__ void __launch_bounds__(128) attn_tc_kernel(const __grid_constant__ CU
                 for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
                 tmem_st_x32(O_t + c * 32, r);
             }
-            tmem_wait_st();
         }
-        fence_proxy_async_smem();
+        tmem_wait_st();
         tc_fence_before();
+        ok = block_wait(bar_v, v_par, p.timeout_ns);  // the block's V has landed
+        if (!ok) break;
+        v_pending = false;
+        v_par ^= 1u;
+        if (tid < KB && kbase + tid >= len) {  // key row past the sequence: zero its V row
+            const uint4 z = make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                reinterpret_cast<uint4*>(sV + tid * 128)[c] = z;
+                reinterpret_cast<uint4*>(sV + KT + tid * 128)[c] = z;
+            }
+            fence_proxy_async_smem();
+        }
         __syncthreads();
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
             for (int k = 0; k < KB / 16; ++k) {
-                const uint64_t a = smem_desc_k128(smem_u32(sP + (k >> 2) * QTILE)) + 2 * (k & 3);
                 const uint64_t bv = smem_desc_mn128(smem_u32(sV + k * 2048), KT, 1024);
-                umma_f16(tmem + 128, a, bv, idesc_o, (kb > 0 || k > 0) ? 1u : 0u);
+                umma_f16_tmem_a(tmem + O_COL, tmem + P_COL + (uint32_t)(k * 8), bv, idesc_o,
+                                (kb > 0 || k > 0) ? 1u : 0u);
             }
-            umma_commit(bar_mma);
+            umma_commit(bar_o);
         }
-        ok = block_wait(bar_mma, mma_phase, p.timeout_ns);
-        mma_phase ^= 1u;
+        ok = block_wait(bar_o, o_phase, p.timeout_ns);
+        o_phase ^= 1u;
         if (!ok) break;
         tc_fence_after();
-        if (kb + 1 < n_kb && tid == 0) issue_kv(kb + 1);
+        if (tid == 0 && kb + 1 < n_kb) issue_v(kb + 1);  // the PV MMAs no longer read V
     }
     if (ok) {
         const float inv = row_ok ? 1.0f / l_i : 0.0f;
@@ -292,7 +325,8 @@ __global__ void __launch_bounds__(128) attn_tc_kernel(const __grid_constant__ CU
         umma_commit(drain);
         mbar_wait_bounded(drain, 0, nullptr, p.timeout_ns);
         if (q_pending) mbar_wait_bounded(bar_q, 0, nullptr, p.timeout_ns);
-        if (kv_pending) mbar_wait_bounded(bar_kv, kv_parity, nullptr, p.timeout_ns);
+        if (k_pending) mbar_wait_bounded(bar_k, k_par, nullptr, p.timeout_ns);
+        if (v_pending) mbar_wait_bounded(bar_v, v_par, nullptr, p.timeout_ns);
     }
     tc_fence_before();
     __syncthreads();
@@ -336,7 +370,7 @@ static CUresult attn_tmap(CUtensorMap* m, int dtype, const void* ptr, int64_t co
                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
-template <typename T, int KB, bool LO>
+template <typename T, bool LO>
 static cudaError_t attn_tc_launch(const void* qkv, const void* qk_lo, int dtype, int H, int qkv_rows,
                                   const AttnTcParams& p, dim3 grid, cudaStream_t st) {
     CUtensorMap tmq, tmk, tmql, tmkl;
@@ -350,10 +384,10 @@ static cudaError_t attn_tc_launch(const void* qkv, const void* qk_lo, int dtype,
     } else {
         tmql = tmq, tmkl = tmk;
     }
-    using C = AttnCfg<KB, LO>;
-    cudaError_t e = prepare_smem((const void*)attn_tc_kernel<T, KB, LO>, C::SMEM);
+    using C = AttnCfg<LO>;
+    cudaError_t e = prepare_smem((const void*)attn_tc_kernel<T, LO>, C::SMEM);
     if (e != cudaSuccess) return e;
-    attn_tc_kernel<T, KB, LO><<<grid, 128, C::SMEM, st>>>(tmq, tmk, tmql, tmkl, p);
+    attn_tc_kernel<T, LO><<<grid, 128, C::SMEM, st>>>(tmq, tmk, tmql, tmkl, p);
     return cudaGetLastError();
 }
 
@@ -369,12 +403,11 @@ cudaError_t launch_attention_tc(int dtype, const void* qkv, const void* qk_lo, v
     p.scale_log2e = (float)(1.4426950408889634 / sqrt((double)AHD));
     p.timeout_ns = timeout_ns;
     dim3 grid((max_len + ATQ - 1) / ATQ, n_heads, batch);
-    // With the low halves, 64-key blocks fit two CTAs per SM; without them 128-key blocks do.
     if (dtype == ENERGON_BF16)
-        return qk_lo ? attn_tc_launch<__nv_bfloat16, KB_LO, true>(qkv, qk_lo, dtype, H, qkv_rows, p, grid, st)
-                     : attn_tc_launch<__nv_bfloat16, 128, false>(qkv, qk_lo, dtype, H, qkv_rows, p, grid, st);
-    return qk_lo ? attn_tc_launch<__half, KB_LO, true>(qkv, qk_lo, dtype, H, qkv_rows, p, grid, st)
-                 : attn_tc_launch<__half, 128, false>(qkv, qk_lo, dtype, H, qkv_rows, p, grid, st);
+        return qk_lo ? attn_tc_launch<__nv_bfloat16, true>(qkv, qk_lo, dtype, H, qkv_rows, p, grid, st)
+                     : attn_tc_launch<__nv_bfloat16, false>(qkv, qk_lo, dtype, H, qkv_rows, p, grid, st);
+    return qk_lo ? attn_tc_launch<__half, true>(qkv, qk_lo, dtype, H, qkv_rows, p, grid, st)
+                 : attn_tc_launch<__half, false>(qkv, qk_lo, dtype, H, qkv_rows, p, grid, st);
 }
 
 }  // namespace energon
