@@ -176,7 +176,7 @@ __global__ void __launch_bounds__(256) ln_rows_generic_kernel(const Tin* __restr
 
 // u = x * g, stats = (rstd, mean * rstd); N elements per step (16-byte vectors when VEC).
 // One warp per row (the row is streamed, nothing of it is kept), eight rows per block:
-// every row of the batch is in flight at once, each lane with four vectors outstanding,
+// every row of the batch is in flight at once, each lane with eight vectors outstanding,
 // and the row statistics need only shuffles.
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(256) ln_fold_kernel(const T* __restrict__ x, const T* __restrict__ g,
@@ -184,7 +184,7 @@ __global__ void __launch_bounds__(256) ln_fold_kernel(const T* __restrict__ x, c
                                                       const int32_t* d_rows, int rows_cap, int H, float eps,
                                                       const int32_t* status, LnGather gth) {
     constexpr int N = VEC ? 16 / sizeof(T) : 1;
-    constexpr int U = 4;
+    constexpr int U = 8;
     if (status_bad(status)) return;
     const int rows = min(*d_rows, rows_cap);
     const int nvec = H / N;
