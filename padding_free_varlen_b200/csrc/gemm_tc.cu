@@ -71,6 +71,9 @@ struct TcParams {
     const float* fold_d;
     void* lo;
     int lo_cols;
+    // the fp32 rows the main drain moves row per lane (the EPI_RES32 residual, the
+    // EPI_RES_OUT32 output) start on 32-byte boundaries: it uses 32-byte accesses
+    int wide32;
 };
 
 // Destination row of packed row `row` (its padded position when the epilogue scatters).
@@ -140,16 +143,39 @@ struct Epi {
     static constexpr int RES_VECS = RES_F32 ? 8 : (RES_T ? 4 : 0);  // 16-byte vectors per 32 columns
 };
 
+// 32-byte global accesses: a lane that owns a row moves whole 32-byte sectors, so a warp
+// instruction touches 32 sectors instead of 32 half sectors (half the requests of 16-byte
+// accesses for the row-per-lane epilogue).
+__device__ __forceinline__ void ld_global32B(const void* a, uint4& lo, uint4& hi) {
+    unsigned long long a0, a1, a2, a3;  // as four 64-bit words
+    asm volatile("ld.global.v4.b64 {%0, %1, %2, %3}, [%4];" : "=l"(a0), "=l"(a1), "=l"(a2), "=l"(a3) : "l"(a));
+    lo = make_uint4((unsigned)a0, (unsigned)(a0 >> 32), (unsigned)a1, (unsigned)(a1 >> 32));
+    hi = make_uint4((unsigned)a2, (unsigned)(a2 >> 32), (unsigned)a3, (unsigned)(a3 >> 32));
+}
+__device__ __forceinline__ void st_global32B(void* a, const float* v) {
+    const unsigned long long w0 = ((unsigned long long)__float_as_uint(v[1]) << 32) | __float_as_uint(v[0]);
+    const unsigned long long w1 = ((unsigned long long)__float_as_uint(v[3]) << 32) | __float_as_uint(v[2]);
+    const unsigned long long w2 = ((unsigned long long)__float_as_uint(v[5]) << 32) | __float_as_uint(v[4]);
+    const unsigned long long w3 = ((unsigned long long)__float_as_uint(v[7]) << 32) | __float_as_uint(v[6]);
+    asm volatile("st.global.v4.b64 [%0], {%1, %2, %3, %4};" ::"l"(a), "l"(w0), "l"(w1), "l"(w2), "l"(w3) : "memory");
+}
+
 // Residual of one row's 32 columns [col0, col0 + 32), read straight from global memory.
-template <typename T, int EPI>
+// WIDE: in 32-byte accesses (the main drain, when the residual rows are 32-byte aligned).
+template <typename T, int EPI, bool WIDE = false>
 __device__ __forceinline__ void load_residual32(const TcParams& p, int row, int col0, bool live, uint4* res) {
     constexpr int NV = Epi<EPI>::RES_VECS;
     if (NV > 0 && live) {
         const size_t eb = Epi<EPI>::RES_F32 ? 4 : sizeof(T);
         const uint4* rp = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.residual) +
                                                          ((size_t)row * p.N + col0) * eb);
+        if constexpr (WIDE && NV % 2 == 0) {
 #pragma unroll
-        for (int q = 0; q < NV; ++q) res[q] = rp[q];
+            for (int q = 0; q < NV; q += 2) ld_global32B(rp + q, res[q], res[q + 1]);
+        } else {
+#pragma unroll
+            for (int q = 0; q < NV; ++q) res[q] = rp[q];
+        }
     }
 }
 
@@ -309,7 +335,7 @@ __device__ __forceinline__ uint32_t stage_off(int row, int chunk) {
 // from the other buffer).  Residuals in the storage type are fetched by TMA into the
 // other buffer one chunk ahead; fp32 residuals are loaded into registers one chunk
 // ahead; fp32 outputs are stored straight from registers, each thread writing whole
-// 128-byte lines of its row.  The accumulator is handed back (arrival on
+// 128-byte lines of its row in 32-byte accesses.  The accumulator is handed back (arrival on
 // `tempty_cluster`) as soon as its last columns are in registers.  Every row of the
 // warp must be valid (rows < M); the warp holding the last valid row takes drain_256
 // instead.  Returns false if a residual copy timed out.
@@ -342,7 +368,10 @@ __device__ __forceinline__ bool drain_256_staged(uint32_t tbase, const TcParams&
     }
     if (TMA_RES) pend = 1u;
     __syncwarp();
-    if (E::RES_F32) load_residual32<T, EPI>(p, row, col_base, true, res[0]);
+    if (E::RES_F32) {
+        if (p.wide32) load_residual32<T, EPI, true>(p, row, col_base, true, res[0]);
+        else load_residual32<T, EPI>(p, row, col_base, true, res[0]);
+    }
     if (RB == 2) {
         tmem_ld_x16(tbase, r[0]);
         tmem_ld_x16(tbase + 16, r[0] + 16);
@@ -355,7 +384,10 @@ __device__ __forceinline__ bool drain_256_staged(uint32_t tbase, const TcParams&
         if (RB == 1) {
             tmem_ld_x16(tbase + c * 32, r[0]);
             tmem_ld_x16(tbase + c * 32 + 16, r[0] + 16);
-            if (c + 1 < CH) load_residual32<T, EPI>(p, row, col_base + (c + 1) * 32, true, res[cur ^ 1]);
+            if (c + 1 < CH) {
+                if (p.wide32) load_residual32<T, EPI, true>(p, row, col_base + (c + 1) * 32, true, res[cur ^ 1]);
+                else load_residual32<T, EPI>(p, row, col_base + (c + 1) * 32, true, res[cur ^ 1]);
+            }
         }
         tmem_wait_ld_regs(r[rc]);
         if (c + 1 < CH) {
@@ -398,9 +430,15 @@ __device__ __forceinline__ bool drain_256_staged(uint32_t tbase, const TcParams&
         float* v = reinterpret_cast<float*>(r[rc]);  // the chunk's values replace its accumulator bits
         epi_math<T, EPI>(v, r[rc], p, col0, fs, TMA_RES ? rt : res[cur]);
         if (E::OUT_F32) {
-            float4* op = reinterpret_cast<float4*>(static_cast<float*>(p.out) + (int64_t)(out_row_base + lane) * p.N + col0);
+            float* op = static_cast<float*>(p.out) + (int64_t)(out_row_base + lane) * p.N + col0;
+            if (p.wide32) {
 #pragma unroll
-            for (int q = 0; q < 8; ++q) op[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                for (int q = 0; q < 4; ++q) st_global32B(op + 8 * q, v + 8 * q);
+            } else {
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    reinterpret_cast<float4*>(op)[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+            }
             continue;
         }
         if (lo) {
@@ -1217,6 +1255,10 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st, char* err, size_t
     p.fold_d = a.fold_d;
     p.lo = a.epilogue == EPI_LN_FOLD ? a.lo : nullptr;
     p.lo_cols = p.lo ? a.lo_cols : 0;
+    {
+        const void* rows32 = a.epilogue == EPI_RES32 ? a.residual : (a.epilogue == EPI_RES_OUT32 ? a.out : nullptr);
+        p.wide32 = rows32 != nullptr && (uintptr_t)rows32 % 32 == 0 && ((size_t)a.N * 4) % 32 == 0 ? 1 : 0;
+    }
     const bool bf = a.dtype == ENERGON_BF16;
     if (a.scatter_cu != nullptr && (single || a.epilogue == EPI_RES_OUT32 || a.epilogue == EPI_LN_FOLD)) {
         if (err) snprintf(err, errlen, "a scattering epilogue needs the CTA-pair path (more than %d rows) and a "

@@ -284,6 +284,36 @@ def test_gemm_wave_tail_cut_does_not_change_rows(oracle_lib, S, lens):
         check_end_to_end(to_f64(out1[b, :n]), ref[j, :n], synth.F16, f"wave-tail layer seq {b}")
 
 
+def test_workspace_offset_by_16_bytes_gives_the_same_rows():
+    """The GEMM epilogues move fp32 rows (the out-projection's output, FFN2's residual) in
+    32-byte accesses when those rows start on 32-byte boundaries and in 16-byte accesses
+    otherwise.  A workspace that starts 16 bytes past a 32-byte boundary takes the second
+    path; the results must be bit-identical to an aligned workspace's."""
+    shape = synth.LayerShape(1024, 8, 2560)
+    H = shape.hidden
+    lengths = np.array([96, 160] * 8, np.int32)
+    B, S = len(lengths), 256
+    x = synth.normal((B, S, H), 33, synth.TID_X, synth.F16)
+    keep = [gpu_layer_weights(shape, 0, 33, synth.F16, NONZERO)]
+    cfg = capi.make_config(H, shape.n_heads, shape.ffn, capi.ENERGON_F16)
+    ws_bytes = capi.energon_workspace_bytes(cfg, B, S)
+    big = torch.empty(ws_bytes + 1024, dtype=torch.uint8, device="cuda")
+    assert big.data_ptr() % 256 == 0
+    d_in = to_device(x, synth.F16)
+    d_len = torch.from_numpy(lengths).cuda()
+    tables = [capi.make_weights(d) for _, d in keep]
+    outs = []
+    for off in (0, 16):
+        ws = big[off:off + ws_bytes]
+        out = torch.empty_like(d_in)
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        capi.energon_stack_forward(cfg, tables, 1, d_in, d_len, B, S, 1, out, st, ws, ws_bytes)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        outs.append(out)
+    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+
+
 def test_prepared_fold_vectors_match_the_per_call_ones(oracle_lib):
     """energon_layer_fold_weights writes c = W_qkv ln1_g and d = b_qkv + W_qkv ln1_b (checked
     against the oracle's linear map); a stack given them returns, bit for bit, what it
