@@ -819,6 +819,16 @@ def cost_table(points, max_b: int, max_s: int):
     return t.tolist()
 
 
+def extend_positions(pool, n: int):
+    """[B, S, H] request rows with at least n positions: a workload padded to fewer positions
+    repeats its own (the values do not change the work); the batches cut from it must have
+    every position their pad length claims."""
+    if pool.shape[1] >= n:
+        return pool
+    reps = (n + pool.shape[1] - 1) // pool.shape[1]
+    return pool.repeat(1, reps, 1)[:, :n].contiguous()
+
+
 def run_batching(capi, synth, cfg, tables, L, tdt, dev, stream, tm: Timer, pool, st):
     """Serves 256 requests (lengths U[1, 256], all queued at once) in batches of at most 64:
     FIFO packing vs the dynamic-programming scheduler (energon_sched_plan), each batch padded
@@ -834,12 +844,14 @@ def run_batching(capi, synth, cfg, tables, L, tdt, dev, stream, tm: Timer, pool,
     arrivals = [0.0] * n_req
     ws_bytes = capi.energon_workspace_bytes(cfg, max_b, max_s)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    pool = extend_positions(pool, max_s)
     nb = pool.shape[0]
     reps = 3
 
     def make_batch(members):
         s_pad = max(lengths[i] for i in members)
         x = torch.stack([pool[i % nb, :s_pad] for i in members]).contiguous()
+        assert x.shape[1] == s_pad
         lens = torch.tensor([lengths[i] for i in members], dtype=torch.int32, device=dev)
         return x, lens, torch.empty_like(x), s_pad
 
@@ -856,6 +868,7 @@ def run_batching(capi, synth, cfg, tables, L, tdt, dev, stream, tm: Timer, pool,
     pts = []
     for b, s_len in COST_SHAPES:
         x = torch.stack([pool[i % nb, :s_len] for i in range(b)]).contiguous()
+        assert x.shape[1] == s_len
         lens = torch.full((b,), s_len, dtype=torch.int32, device=dev)
         out = torch.empty_like(x)
         f = lambda: capi.energon_stack_forward(cfg, tables, L, x, lens, b, s_len, 0, out, st, ws, ws_bytes, stream)

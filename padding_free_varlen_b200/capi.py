@@ -125,6 +125,16 @@ def _dev(x, what: str) -> int:
     return x.data_ptr()
 
 
+def _need(x, nbytes: int, what: str) -> None:
+    """A tensor argument must hold at least the bytes the call will touch (the C ABI takes
+    the sizes on trust); raw integer addresses are the caller's responsibility."""
+    if isinstance(x, torch.Tensor) and x.numel() * x.element_size() < nbytes:
+        raise ValueError(f"{what}: {x.numel() * x.element_size()} bytes, the call needs {nbytes}")
+
+
+_ELEM_BYTES = {0: 4, 1: 2, 2: 2}  # ENERGON_F32, ENERGON_F16, ENERGON_BF16
+
+
 def _stream(s) -> int:
     if s is None:
         return torch.cuda.current_stream().cuda_stream
@@ -147,12 +157,17 @@ def energon_set_wait_timeout_us(timeout_us: int) -> None:
 
 
 def energon_rce_offsets(lengths, batch, pad_len, cu_seqlens, d_status, stream=None) -> None:
+    _need(lengths, 4 * batch, "lengths")
+    _need(cu_seqlens, 4 * (batch + 1), "cu_seqlens")
     _check(load().energon_rce_offsets(_dev(lengths, "lengths"), batch, pad_len, _dev(cu_seqlens, "cu_seqlens"),
                                       _dev(d_status, "d_status"), _stream(stream)), "energon_rce_offsets")
 
 
 def energon_rce_remove_padding(padded, cu_seqlens, batch, pad_len, hidden, elem_bytes, packed,
                                stream=None) -> None:
+    _need(padded, batch * pad_len * hidden * elem_bytes, "padded")
+    _need(packed, batch * pad_len * hidden * elem_bytes, "packed")
+    _need(cu_seqlens, 4 * (batch + 1), "cu_seqlens")
     _check(load().energon_rce_remove_padding(_dev(padded, "padded"), _dev(cu_seqlens, "cu_seqlens"), batch,
                                              pad_len, hidden, elem_bytes, _dev(packed, "packed"), _stream(stream)),
            "energon_rce_remove_padding")
@@ -160,6 +175,8 @@ def energon_rce_remove_padding(padded, cu_seqlens, batch, pad_len, hidden, elem_
 
 def energon_rce_rebuild_padding(packed, cu_seqlens, batch, pad_len, hidden, elem_bytes, padded,
                                 stream=None) -> None:
+    _need(padded, batch * pad_len * hidden * elem_bytes, "padded")
+    _need(cu_seqlens, 4 * (batch + 1), "cu_seqlens")
     _check(load().energon_rce_rebuild_padding(_dev(packed, "packed"), _dev(cu_seqlens, "cu_seqlens"), batch,
                                               pad_len, hidden, elem_bytes, _dev(padded, "padded"), _stream(stream)),
            "energon_rce_rebuild_padding")
@@ -167,6 +184,8 @@ def energon_rce_rebuild_padding(packed, cu_seqlens, batch, pad_len, hidden, elem
 
 def energon_rce_transpose_padding_rebuild(packed, cu_seqlens, batch, pad_len, parts, n_heads, head_dim, elem_bytes,
                                           heads, stream=None) -> None:
+    _need(heads, parts * batch * n_heads * pad_len * head_dim * elem_bytes, "heads")
+    _need(cu_seqlens, 4 * (batch + 1), "cu_seqlens")
     _check(load().energon_rce_transpose_padding_rebuild(_dev(packed, "packed"), _dev(cu_seqlens, "cu_seqlens"), batch,
                                                         pad_len, parts, n_heads, head_dim, elem_bytes,
                                                         _dev(heads, "heads"), _stream(stream)),
@@ -175,6 +194,8 @@ def energon_rce_transpose_padding_rebuild(packed, cu_seqlens, batch, pad_len, pa
 
 def energon_rce_transpose_padding_remove(heads, cu_seqlens, batch, pad_len, parts, n_heads, head_dim, elem_bytes,
                                          packed, stream=None) -> None:
+    _need(heads, parts * batch * n_heads * pad_len * head_dim * elem_bytes, "heads")
+    _need(cu_seqlens, 4 * (batch + 1), "cu_seqlens")
     _check(load().energon_rce_transpose_padding_remove(_dev(heads, "heads"), _dev(cu_seqlens, "cu_seqlens"), batch,
                                                        pad_len, parts, n_heads, head_dim, elem_bytes,
                                                        _dev(packed, "packed"), _stream(stream)),
@@ -185,6 +206,9 @@ def energon_rce_remove_padding_noalloc(padded, lengths, batch, pad_len, hidden, 
                                        stream=None) -> None:
     """Offsets + transpose_padding_remove with the offsets kept in the library's own
     fixed scratch array: for callers that cannot allocate (batch <= ENERGON_NOALLOC_MAX_BATCH)."""
+    _need(padded, batch * pad_len * hidden * elem_bytes, "padded")
+    _need(packed, batch * pad_len * hidden * elem_bytes, "packed")
+    _need(lengths, 4 * batch, "lengths")
     _check(load().energon_rce_remove_padding_noalloc(_dev(padded, "padded"), _dev(lengths, "lengths"), batch, pad_len,
                                                      hidden, elem_bytes, _dev(packed, "packed"),
                                                      _dev(d_status, "d_status"), _stream(stream)),
@@ -197,6 +221,11 @@ def energon_workspace_bytes(cfg: energon_layer_config, batch: int, pad_len: int)
 
 def energon_layer_forward(cfg, weights, x_packed, cu_seqlens, batch, max_len, y_packed, d_status, workspace,
                           ws_bytes, stream=None) -> None:
+    rows_bytes = batch * max_len * cfg.hidden * _ELEM_BYTES.get(cfg.dtype, 4)
+    _need(x_packed, rows_bytes, "x_packed")
+    _need(y_packed, rows_bytes, "y_packed")
+    _need(cu_seqlens, 4 * (batch + 1), "cu_seqlens")
+    _need(workspace, ws_bytes, "workspace")
     _check(load().energon_layer_forward(ctypes.byref(cfg), ctypes.byref(weights), _dev(x_packed, "x_packed"),
                                         _dev(cu_seqlens, "cu_seqlens"), batch, max_len, _dev(y_packed, "y_packed"),
                                         _dev(d_status, "d_status"), _dev(workspace, "workspace"), ws_bytes,
@@ -205,6 +234,11 @@ def energon_layer_forward(cfg, weights, x_packed, cu_seqlens, batch, max_len, y_
 
 def energon_stack_forward(cfg, layers, n_layers, padded_in, lengths, batch, pad_len, remove_padding, padded_out,
                           d_status, workspace, ws_bytes, stream=None) -> None:
+    rows_bytes = batch * pad_len * cfg.hidden * _ELEM_BYTES.get(cfg.dtype, 4)
+    _need(padded_in, rows_bytes, "padded_in")
+    _need(padded_out, rows_bytes, "padded_out")
+    _need(lengths, 4 * batch, "lengths")
+    _need(workspace, ws_bytes, "workspace")
     arr = layers if isinstance(layers, ctypes.Array) else (energon_layer_weights * max(1, len(layers)))(*layers)
     _check(load().energon_stack_forward(ctypes.byref(cfg), arr, n_layers, _dev(padded_in, "padded_in"),
                                         _dev(lengths, "lengths"), batch, pad_len, int(remove_padding),

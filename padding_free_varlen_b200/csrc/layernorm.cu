@@ -237,6 +237,59 @@ __global__ void __launch_bounds__(256) ln_fold_kernel(const T* __restrict__ x, c
     }
 }
 
+// The same outputs with one block of 256 threads per row and the row in registers, for
+// batches of few rows: a warp streaming a 12288-element row alone waits on a chain of
+// dependent loads (tens of microseconds at 32 rows), where a block has its whole row in
+// flight at once.  VPT 16-byte vectors per thread (the row has H / N of them, at most
+// 256 * VPT).
+template <typename T, int VPT>
+__global__ void __launch_bounds__(256) ln_fold_rows_kernel(const T* __restrict__ x, const T* __restrict__ g,
+                                                           T* __restrict__ u, float2* __restrict__ stats,
+                                                           const int32_t* d_rows, int rows_cap, int H, float eps,
+                                                           const int32_t* status, LnGather gth) {
+    constexpr int N = 16 / sizeof(T);
+    __shared__ float2 red[32];
+    if (status_bad(status)) return;
+    const int rows = min(*d_rows, rows_cap);
+    const int nvec = H / N;
+    T* copy = static_cast<T*>(gth.copy);
+    for (int r = blockIdx.x; r < rows; r += gridDim.x) {
+        const int64_t src = ln_src_row(gth, r);
+        if (src < 0) continue;  // the same for every thread of the block
+        const T* xr = x + src * H;
+        T* ur = u + (int64_t)r * H;
+        T* cr = copy ? copy + (int64_t)r * H : nullptr;
+        const float x0 = to_f(xr[0]);
+        Pack<T, N> xv[VPT];
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            const int idx = i * blockDim.x + threadIdx.x;
+            if (idx < nvec) xv[i] = *reinterpret_cast<const Pack<T, N>*>(xr + (int64_t)idx * N);
+        }
+        float2 s = make_float2(0.0f, 0.0f);
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            const int idx = i * blockDim.x + threadIdx.x;
+            if (idx >= nvec) continue;
+            const int64_t e = (int64_t)idx * N;
+            if (cr) *reinterpret_cast<Pack<T, N>*>(cr + e) = xv[i];
+            float gv[N], o[N];
+            load_f_ldg<T, N>(g + e, gv);
+#pragma unroll
+            for (int j = 0; j < N; ++j) {
+                const float v = to_f(xv[i].v[j]);
+                const float d = v - x0;
+                s.x += d;
+                s.y = fmaf(d, d, s.y);
+                o[j] = v * gv[j];
+            }
+            store_f<T, N>(ur + e, o);
+        }
+        const float2 mi = row_stats(x0, block_sum2(s, red), H, eps);
+        if (threadIdx.x == 0) stats[r] = make_float2(mi.y, mi.x * mi.y);
+    }
+}
+
 // c[n] = sum_k g[k] W[n][k], d[n] = bias[n] + sum_k beta[k] W[n][k].  A block of 256
 // threads owns RPB consecutive rows of W; thread t takes the 16-byte vectors t, t + 256,
 // ... of every row, two vector steps at a time, so each thread has 2 * (RPB + 2) loads in
@@ -324,6 +377,9 @@ static int resident_blocks(K kernel) {
     });
 }
 
+// Buffers of at most this many rows take the block-per-row form of the folded LayerNorm.
+constexpr int LN_FOLD_BLOCK_ROWS = 512;
+
 static int row_grid(int rows_cap, int resident) {
     return rows_cap < resident ? (rows_cap > 0 ? rows_cap : 1) : resident;
 }
@@ -384,6 +440,19 @@ static cudaError_t ln_fold_dispatch(const void* x, const void* g, void* u, float
                                     cudaStream_t st) {
     constexpr int N = 16 / sizeof(T);
     const uintptr_t al = (uintptr_t)x | (uintptr_t)g | (uintptr_t)u | (uintptr_t)gth.copy;
+    const int vpt = (H / N + 255) / 256;
+    if (H % N == 0 && al % 16 == 0 && rows_cap <= LN_FOLD_BLOCK_ROWS && vpt <= 8) {
+        // few rows: a block per row
+        auto launch = [&](auto k) {
+            k<<<row_grid(rows_cap, resident_blocks(k)), 256, 0, st>>>((const T*)x, (const T*)g, (T*)u, stats, d_rows,
+                                                                      rows_cap, H, eps, status, gth);
+        };
+        if (vpt <= 2) launch(ln_fold_rows_kernel<T, 2>);
+        else if (vpt <= 4) launch(ln_fold_rows_kernel<T, 4>);
+        else if (vpt <= 6) launch(ln_fold_rows_kernel<T, 6>);
+        else launch(ln_fold_rows_kernel<T, 8>);
+        return cudaGetLastError();
+    }
     // eight rows (warps) per block, as many blocks as the rows need or the GPU holds
     const int row_blocks = (rows_cap + 7) / 8;
     if (H % N == 0 && al % 16 == 0) {

@@ -77,3 +77,31 @@ def test_batching_cost_table_interpolates_the_measured_points():
     # monotone in the padded token count, as the measured points are
     flat = sorted(((b + 1) * (s + 1), t[b][s]) for b in range(64) for s in range(256))
     assert all(flat[i][1] <= flat[i + 1][1] + 1e-15 for i in range(len(flat) - 1))
+
+
+def test_batching_pool_has_every_position_a_batch_claims():
+    """The dynamic-batching section cuts batches of up to 256 positions from the workload's
+    padded input; a workload padded to 64 positions (gpt3_layer) repeats its positions so that
+    no batch is shorter than the pad length passed with it."""
+    import torch
+    pool = torch.arange(2 * 64 * 3, dtype=torch.float32).reshape(2, 64, 3)
+    ext = bench.extend_positions(pool, 256)
+    assert ext.shape == (2, 256, 3) and ext.is_contiguous()
+    assert torch.equal(ext[:, :64], pool) and torch.equal(ext[:, 64:128], pool)
+    assert bench.extend_positions(pool, 64) is pool
+
+
+def test_binding_refuses_tensors_smaller_than_the_call_needs():
+    """The C ABI takes sizes on trust; the binding checks every tensor argument against the
+    bytes the call will touch before anything reaches a kernel."""
+    import torch
+    from padding_free_varlen_b200 import capi
+    cfg = capi.make_config(256, 2, 1024, capi.ENERGON_F16)
+    w = capi.energon_layer_weights(*([0] * 13))
+    small = torch.zeros((2, 4, 256), dtype=torch.float16)          # 4 positions, the call claims 8
+    with pytest.raises(ValueError, match="padded_in"):
+        capi.energon_stack_forward(cfg, [w], 1, small, torch.zeros(2, dtype=torch.int32), 2, 8, 1, small,
+                                   torch.zeros(1, dtype=torch.int32), torch.zeros(1, dtype=torch.uint8), 1, stream=0)
+    with pytest.raises(ValueError, match="packed"):
+        capi.energon_rce_remove_padding(torch.zeros((2, 8, 16), dtype=torch.float16), torch.zeros(3, dtype=torch.int32),
+                                        2, 8, 16, 2, torch.zeros((8, 16), dtype=torch.float16), stream=0)
