@@ -823,11 +823,18 @@ __global__ void __launch_bounds__(PairCfg<MT, BN>::THREADS, 1)
     // shapes at T = 4096 and ran about 1 % faster; L2 eviction-priority hints made the
     // kernel 10 % slower.
     const int group = 8;
-    // unit u -> pair tile t, its row tiles [i0, i1) and column half h (-1: all columns)
+    // unit u -> pair tile t, its row tiles [i0, i1) and column half h (-1: all columns).  A
+    // full tile of the last pair row keeps only the row tiles that hold rows below M (an odd
+    // number of 256-row tiles leaves the last pair row half empty: its MMAs are skipped).
     auto unit_of = [&](int u, int& t, int& i0, int& i1, int& h) {
         h = -1;
         if (u < full_units) {
             t = u, i0 = 0, i1 = MT;
+            if (MT > 1 && num_m % MT != 0) {
+                int mt_, n_;
+                tile_coords(t, num_mt, num_n, group, 0, mt_, n_);
+                if (mt_ == num_mt - 1) i1 = num_m - mt_ * MT;
+            }
         } else {
             const int v = u - full_units;
             if (split == 2) {

@@ -258,15 +258,17 @@ def test_stack_packed_equals_padded_and_oracle(oracle_lib, dtype):
                              f"alone vs batch seq {b}")
 
 
-@pytest.mark.parametrize("S,lens", [(512, [192, 320]), (256, [96, 160])])
+@pytest.mark.parametrize("S,lens", [(512, [192, 320]), (256, [96, 160]), (256, [240, 240])])
 def test_gemm_wave_tail_cut_does_not_change_rows(oracle_lib, S, lens):
     """Hidden 1024, FFN 2560, 16 sequences.  On 148 SMs (74 CTA pairs) the last, partly
     filled round of 512 x 256 pair tiles is cut into half units (one row tile) or quarter
     units (one row tile, 128 columns) depending on how many tiles it holds: with 4096
     valid tokens the packed QKV and FFN1 GEMMs (96 and 80 tiles) cut their tail in halves;
     with 2048 the out-projection and FFN2 (16 tiles) and FFN1 (40) cut it in quarters.
-    The padded runs (twice the rows) cut differently or not at all.  Valid rows must agree
-    bit for bit across the three modes, and match the oracle."""
+    With 3840 (15 row tiles of 256) the last pair row holds one row tile, and the full
+    tiles of that row skip the empty one.  The padded runs (more rows) cut differently or
+    not at all.  Valid rows must agree bit for bit across the three modes, and match the
+    oracle."""
     shape = synth.LayerShape(1024, 8, 2560)
     B = 16
     lengths = np.array(lens * 8, np.int32)
