@@ -1,10 +1,11 @@
 """Thin ctypes binding of ``libenergon_rce.so`` (the C ABI in ``include/energon_rce.h``).
 
 Each function has the name of the C entry point it calls and only marshals
-arguments: torch tensors become device pointers, streams become
-``cudaStream_t`` handles, and a nonzero return code raises ``EnergonError``
-with the library's message.  Every step of the path runs in the CUDA
-library; if it is missing, the first call fails loudly.
+arguments: torch tensors become device pointers (after a check that each
+holds the bytes the call will touch, since the C ABI takes sizes on trust),
+streams become ``cudaStream_t`` handles, and a nonzero return code raises
+``EnergonError`` with the library's message.  Every step of the path runs in
+the CUDA library; if it is missing, the first call fails loudly.
 """
 from __future__ import annotations
 
