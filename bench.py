@@ -252,15 +252,15 @@ def gemm_device_code_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def traffic_from_profile() -> int | None:
-    """DRAM bytes per launch of the GEMM kernel from the committed ncu summary, if the GEMM's
-    device code has not changed since the counters were taken."""
+def traffic_from_profile(workload: str) -> int | None:
+    """DRAM bytes per launch of the GEMM kernel from the committed ncu summary, if it was taken
+    on this workload's launch configuration and the GEMM's device code has not changed since."""
     path = os.path.join(ROOT, "profiles", "gemm_tc_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         d = json.load(f)
-    if d.get("device_code_sha256_16") != gemm_device_code_hash():
+    if d.get("device_code_sha256_16") != gemm_device_code_hash() or d.get("workload") != workload:
         return None
     return d.get("dram_bytes_per_launch_scaled")
 
@@ -539,7 +539,7 @@ def bench_stack(args, dist: Dist, wl, dev, stream, peaks: dict, want_cpu: bool, 
     res["traced_pass"] = {"ms_per_step": ms_traced / args.steps,
                           "note": "per-kernel shares and the roofline come from this pass; the headline is untraced"}
     res["gpu_launches"] = sum(v[0] for v in trace.values())    # the same K steps as the headline
-    res["roofline"] = gemm_roofline(H, T, e, g_launch, g_ms, peaks, traffic_from_profile())
+    res["roofline"] = gemm_roofline(H, T, e, g_launch, g_ms, peaks, traffic_from_profile(wl.name))
     res["step_roofline"] = step_roofline(H, L, lengths, e, ms / args.steps, peaks)
     aux = {}
     lo = 2 if e == 2 else 0   # the low halves of Q and K (16-bit types)

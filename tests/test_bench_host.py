@@ -105,3 +105,16 @@ def test_binding_refuses_tensors_smaller_than_the_call_needs():
     with pytest.raises(ValueError, match="packed"):
         capi.energon_rce_remove_padding(torch.zeros((2, 8, 16), dtype=torch.float16), torch.zeros(3, dtype=torch.int32),
                                         2, 8, 16, 2, torch.zeros((8, 16), dtype=torch.float16), stream=0)
+
+
+def test_gemm_traffic_record_applies_to_its_own_workload_only(monkeypatch):
+    """The committed DRAM count was taken on one launch configuration (the half-padded GPT-3
+    stack); the roofline of another workload must not report it."""
+    import json
+    with open(os.path.join(os.path.dirname(os.path.abspath(bench.__file__)), "profiles", "gemm_tc_traffic.json")) as f:
+        rec = json.load(f)
+    monkeypatch.setattr(bench, "gemm_device_code_hash", lambda: rec["device_code_sha256_16"])
+    assert bench.traffic_from_profile(rec["workload"]) == rec["dram_bytes_per_launch_scaled"]
+    assert bench.traffic_from_profile("gpt3_stack_dynbatch") is None
+    monkeypatch.setattr(bench, "gemm_device_code_hash", lambda: "0" * 16)
+    assert bench.traffic_from_profile(rec["workload"]) is None
