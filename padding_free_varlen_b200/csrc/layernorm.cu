@@ -9,8 +9,10 @@
 //    One thread block per row; each thread keeps its slice of the row in
 //    registers, so the row is read from HBM once and written once.
 //  - ln_fold_kernel: the LayerNorm before the QKV projection, folded into that
-//    GEMM (one warp per row; the row is streamed, not kept).  It writes u = x * g (rounded to the storage type: exact when g is 1)
-//    and the row statistics (rstd, mean * rstd); the GEMM's epilogue finishes
+//    GEMM (one warp per row; the row is streamed, not kept; buffers of at most
+//    512 rows take ln_fold_rows_kernel, a block per row with the row in
+//    registers).  It writes u = x * g (rounded to the storage type: exact when
+//    g is 1) and the row statistics (rstd, mean * rstd); the GEMM's epilogue finishes
 //    LN(x) W^T + b = rstd (u W^T) - mean rstd c + d with c = W g, d = b + W beta
 //    (ln_fold_weights_kernel).  The tensor cores then see the layer input
 //    itself instead of a rounded normalisation of it, which the attention
