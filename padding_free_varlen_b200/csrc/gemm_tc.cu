@@ -6,7 +6,10 @@
 // bias + GELU and bias + residual steps that follow the MLP GEMMs, fused here
 // into the epilogue instead of separate passes over HBM).
 //
-// Design (one CTA per SM, persistent):
+// Two persistent kernels.  gemm_tc2_kernel, for buffers of more than 128 rows,
+// runs on CTA pairs (cta_group::2) with 512 x 256 pair tiles; it is described
+// before its definition below.  gemm_tc_kernel, for buffers of at most 128 rows
+// (the weight-streaming case, with split K), is the single-CTA form:
 //   - 128 x 256 output tiles, K consumed 64 elements (128 bytes) at a time.
 //   - warp 0: TMA producer.  A [rows, K] and W [N, K] tiles land in a 4-stage
 //     shared-memory ring (128-byte swizzle), completion counted on mbarriers.
