@@ -18,6 +18,8 @@
 //         (columns 64..95, two keys per column)
 //   MMA   O += P V with P read from TMEM and V from shared memory as an MN-major
 //         operand (no transpose), into TMEM columns 128..255
+//   out   O / l staged in the Q buffer and stored by TMA (a full tile) or row by row with
+//         whole 256-byte rows per half warp (a partial tile)
 // P never touches shared memory, so the K buffer is free as soon as the S MMAs
 // are done: the next block's K is fetched while this block's softmax runs, and
 // the next block's V while the next S and softmax run.  A CTA holds 112 KiB of
@@ -99,7 +101,8 @@ template <typename T, bool LO>
 __global__ void __launch_bounds__(128) attn_tc_kernel(const __grid_constant__ CUtensorMap tmq,
                                                       const __grid_constant__ CUtensorMap tmk,
                                                       const __grid_constant__ CUtensorMap tmql,
-                                                      const __grid_constant__ CUtensorMap tmkl, const AttnTcParams p) {
+                                                      const __grid_constant__ CUtensorMap tmkl,
+                                                      const __grid_constant__ CUtensorMap tmo, const AttnTcParams p) {
     using C = AttnCfg<LO>;
     constexpr int KT = KTILE;
     extern __shared__ uint8_t smem_raw[];
@@ -300,23 +303,42 @@ __global__ void __launch_bounds__(128) attn_tc_kernel(const __grid_constant__ CU
         if (tid == 0 && kb + 1 < n_kb) issue_v(kb + 1);  // the PV MMAs no longer read V
     }
     if (ok) {
+        // O, normalised and rounded, staged in the Q buffer (no MMA reads it any more) in the
+        // 128-byte swizzle; a tile whose 128 rows are all valid leaves with two TMA stores, a
+        // partial one row by row, 16 lanes x 16 bytes per row (whole 256-byte rows per
+        // instruction instead of one row per lane)
         const float inv = row_ok ? 1.0f / l_i : 0.0f;
-        T* orow = static_cast<T*>(p.out) + (int64_t)(start + q) * p.H + j * AHD;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
             tmem_ld_x32(O_t + c * 32, r);
             tmem_wait_ld();
-            if (row_ok) {
-                uint4* op = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    uint4 w;
-                    w.x = pack2<T>(__uint_as_float(r[8 * g + 0]) * inv, __uint_as_float(r[8 * g + 1]) * inv);
-                    w.y = pack2<T>(__uint_as_float(r[8 * g + 2]) * inv, __uint_as_float(r[8 * g + 3]) * inv);
-                    w.z = pack2<T>(__uint_as_float(r[8 * g + 4]) * inv, __uint_as_float(r[8 * g + 5]) * inv);
-                    w.w = pack2<T>(__uint_as_float(r[8 * g + 6]) * inv, __uint_as_float(r[8 * g + 7]) * inv);
-                    op[g] = w;
-                }
+            for (int g = 0; g < 4; ++g) {
+                uint4 w;
+                w.x = pack2<T>(__uint_as_float(r[8 * g + 0]) * inv, __uint_as_float(r[8 * g + 1]) * inv);
+                w.y = pack2<T>(__uint_as_float(r[8 * g + 2]) * inv, __uint_as_float(r[8 * g + 3]) * inv);
+                w.z = pack2<T>(__uint_as_float(r[8 * g + 4]) * inv, __uint_as_float(r[8 * g + 5]) * inv);
+                w.w = pack2<T>(__uint_as_float(r[8 * g + 6]) * inv, __uint_as_float(r[8 * g + 7]) * inv);
+                const int ch = (c & 1) * 4 + g;
+                *reinterpret_cast<uint4*>(sQ + (c >> 1) * QTILE + tid * 128 + ((ch ^ (tid & 7)) << 4)) = w;
+            }
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+        const int rows = min(ATQ, len - q0);
+        if (rows == ATQ) {
+            if (tid == 0) {
+                tma_store_2d(&tmo, sQ, j * AHD, start + q0);
+                tma_store_2d(&tmo, sQ + QTILE, j * AHD + 64, start + q0);
+                bulk_commit();
+                bulk_wait_read<0>();  // the buffer stays until the stores have read it
+            }
+        } else {
+            const int lane = tid & 31, k = lane & 15;
+            for (int rr = warp * 2 + (lane >> 4); rr < rows; rr += 8) {
+                const uint4 w =
+                    *reinterpret_cast<const uint4*>(sQ + (k >> 3) * QTILE + rr * 128 + (((k & 7) ^ (rr & 7)) << 4));
+                reinterpret_cast<uint4*>(static_cast<T*>(p.out) + (int64_t)(start + q0 + rr) * p.H + j * AHD)[k] = w;
             }
         }
     } else if (tid == 0) {
@@ -384,10 +406,12 @@ static cudaError_t attn_tc_launch(const void* qkv, const void* qk_lo, int dtype,
     } else {
         tmql = tmq, tmkl = tmk;
     }
+    CUtensorMap tmo;  // the output [rows, H], 128-row boxes
+    if (attn_tmap(&tmo, dtype, p.out, H, qkv_rows, ATQ) != CUDA_SUCCESS) return cudaErrorInvalidValue;
     using C = AttnCfg<LO>;
     cudaError_t e = prepare_smem((const void*)attn_tc_kernel<T, LO>, C::SMEM);
     if (e != cudaSuccess) return e;
-    attn_tc_kernel<T, LO><<<grid, 128, C::SMEM, st>>>(tmq, tmk, tmql, tmkl, p);
+    attn_tc_kernel<T, LO><<<grid, 128, C::SMEM, st>>>(tmq, tmk, tmql, tmkl, tmo, p);
     return cudaGetLastError();
 }
 
