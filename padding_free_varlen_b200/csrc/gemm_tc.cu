@@ -337,8 +337,8 @@ __device__ __forceinline__ uint32_t stage_off(int row, int chunk) {
 // buffer -> one TMA store of the 32 x 32 box (and, for the low halves, a second box
 // from the other buffer).  Residuals in the storage type are fetched by TMA into the
 // other buffer one chunk ahead; fp32 residuals are loaded into registers one chunk
-// ahead; fp32 outputs are stored straight from registers, each thread writing whole
-// 128-byte lines of its row in 32-byte accesses.  The accumulator is handed back (arrival on
+// ahead; fp32 outputs go out through the buffer the chunk's residual has just left, 16
+// columns (one 32 x 16 fp32 box, 64-byte rows) per TMA store.  The accumulator is handed back (arrival on
 // `tempty_cluster`) as soon as its last columns are in registers.  Every row of the
 // warp must be valid (rows < M); the warp holding the last valid row takes drain_256
 // instead.  Returns false if a residual copy timed out.
@@ -406,6 +406,7 @@ __device__ __forceinline__ bool drain_256_staged(uint32_t tbase, const TcParams&
         const int col0 = col_base + c * 32;
         if (TMA_RES && c + 1 < CH) {
             if (lane == 0) {
+                if (E::OUT_F32) bulk_wait_read<0>();  // the previous chunk's output stores used that buffer
                 mbar_arrive_expect_tx(&rbar[cur ^ 1], 32 * 64);
                 tma_load_2d(sbuf + (cur ^ 1) * 2048, tmR, &rbar[cur ^ 1], col0 + 32, row_base);
             }
@@ -433,14 +434,25 @@ __device__ __forceinline__ bool drain_256_staged(uint32_t tbase, const TcParams&
         float* v = reinterpret_cast<float*>(r[rc]);  // the chunk's values replace its accumulator bits
         epi_math<T, EPI>(v, r[rc], p, col0, fs, TMA_RES ? rt : res[cur]);
         if (E::OUT_F32) {
-            float* op = static_cast<float*>(p.out) + (int64_t)(out_row_base + lane) * p.N + col0;
-            if (p.wide32) {
+            // this chunk's residual has been read out of buf: it takes the fp32 output, 16
+            // columns (64-byte rows) at a time, each half one TMA store
 #pragma unroll
-                for (int q = 0; q < 4; ++q) st_global32B(op + 8 * q, v + 8 * q);
-            } else {
+            for (int hh = 0; hh < 2; ++hh) {
+                if (hh == 1) {
+                    if (lane == 0) bulk_wait_read<0>();
+                    __syncwarp();
+                }
 #pragma unroll
-                for (int q = 0; q < 8; ++q)
-                    reinterpret_cast<float4*>(op)[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<float4*>(buf + stage_off(lane, q)) =
+                        make_float4(v[16 * hh + 4 * q], v[16 * hh + 4 * q + 1], v[16 * hh + 4 * q + 2],
+                                    v[16 * hh + 4 * q + 3]);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(tmO, buf, col0 + 16 * hh, out_row_base);
+                    bulk_commit();
+                }
             }
             continue;
         }
@@ -1121,6 +1133,19 @@ static CUresult make_tmap_io(CUtensorMap* m, int dtype, const void* ptr, int64_t
               CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
+// fp32 [rows, N] in 16 x 32 boxes, 64-byte swizzle (the staging buffers' layout).
+static CUresult make_tmap_f32(CUtensorMap* m, const void* ptr, int64_t N, int64_t rows) {
+    auto fn = encode_fn();
+    if (!fn) return CUDA_ERROR_NOT_FOUND;
+    cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)N * 4};
+    cuuint32_t box[2] = {16, 32};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
 // Single-CTA tiles for a GEMM whose rows fit in one 128-row tile (the skinny,
 // weight-streaming case): more CTAs stream weights than with 256-row pair tiles.
 static bool use_single_cta(const GemmArgs& a) { return a.M_cap <= TBM; }
@@ -1293,7 +1318,7 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st, char* err, size_t
         CUresult r3 = CUDA_SUCCESS, r4 = CUDA_SUCCESS, r5 = CUDA_SUCCESS;
         if (a.epilogue == EPI_RES_OUT32) {
             r4 = make_tmap_io(&tr, a.dtype, a.residual, a.N, a.M_cap);
-            to = tr;
+            r3 = make_tmap_f32(&to, a.out, a.N, a.M_cap);
         } else {
             r3 = make_tmap_io(&to, a.dtype, a.out, a.N, out_rows);
             tr = to;
