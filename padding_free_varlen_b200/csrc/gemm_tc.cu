@@ -74,8 +74,8 @@ struct TcParams {
     const float* fold_d;
     void* lo;
     int lo_cols;
-    // the fp32 rows the main drain moves row per lane (the EPI_RES32 residual, the
-    // EPI_RES_OUT32 output) start on 32-byte boundaries: it uses 32-byte accesses
+    // the fp32 residual rows the main drain reads row per lane (EPI_RES32) start on 32-byte
+    // boundaries: it uses 32-byte loads
     int wide32;
 };
 
@@ -146,21 +146,14 @@ struct Epi {
     static constexpr int RES_VECS = RES_F32 ? 8 : (RES_T ? 4 : 0);  // 16-byte vectors per 32 columns
 };
 
-// 32-byte global accesses: a lane that owns a row moves whole 32-byte sectors, so a warp
+// 32-byte global loads: a lane that owns a row reads whole 32-byte sectors, so a warp
 // instruction touches 32 sectors instead of 32 half sectors (half the requests of 16-byte
-// accesses for the row-per-lane epilogue).
+// loads for the row-per-lane fp32 residual).
 __device__ __forceinline__ void ld_global32B(const void* a, uint4& lo, uint4& hi) {
     unsigned long long a0, a1, a2, a3;  // as four 64-bit words
     asm volatile("ld.global.v4.b64 {%0, %1, %2, %3}, [%4];" : "=l"(a0), "=l"(a1), "=l"(a2), "=l"(a3) : "l"(a));
     lo = make_uint4((unsigned)a0, (unsigned)(a0 >> 32), (unsigned)a1, (unsigned)(a1 >> 32));
     hi = make_uint4((unsigned)a2, (unsigned)(a2 >> 32), (unsigned)a3, (unsigned)(a3 >> 32));
-}
-__device__ __forceinline__ void st_global32B(void* a, const float* v) {
-    const unsigned long long w0 = ((unsigned long long)__float_as_uint(v[1]) << 32) | __float_as_uint(v[0]);
-    const unsigned long long w1 = ((unsigned long long)__float_as_uint(v[3]) << 32) | __float_as_uint(v[2]);
-    const unsigned long long w2 = ((unsigned long long)__float_as_uint(v[5]) << 32) | __float_as_uint(v[4]);
-    const unsigned long long w3 = ((unsigned long long)__float_as_uint(v[7]) << 32) | __float_as_uint(v[6]);
-    asm volatile("st.global.v4.b64 [%0], {%1, %2, %3, %4};" ::"l"(a), "l"(w0), "l"(w1), "l"(w2), "l"(w3) : "memory");
 }
 
 // Residual of one row's 32 columns [col0, col0 + 32), read straight from global memory.
@@ -1291,7 +1284,7 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st, char* err, size_t
     p.lo = a.epilogue == EPI_LN_FOLD ? a.lo : nullptr;
     p.lo_cols = p.lo ? a.lo_cols : 0;
     {
-        const void* rows32 = a.epilogue == EPI_RES32 ? a.residual : (a.epilogue == EPI_RES_OUT32 ? a.out : nullptr);
+        const void* rows32 = a.epilogue == EPI_RES32 ? a.residual : nullptr;
         p.wide32 = rows32 != nullptr && (uintptr_t)rows32 % 32 == 0 && ((size_t)a.N * 4) % 32 == 0 ? 1 : 0;
     }
     const bool bf = a.dtype == ENERGON_BF16;

@@ -287,10 +287,10 @@ def test_gemm_wave_tail_cut_does_not_change_rows(oracle_lib, S, lens):
 
 
 def test_workspace_offset_by_16_bytes_gives_the_same_rows():
-    """The GEMM epilogues move fp32 rows (the out-projection's output, FFN2's residual) in
-    32-byte accesses when those rows start on 32-byte boundaries and in 16-byte accesses
-    otherwise.  A workspace that starts 16 bytes past a 32-byte boundary takes the second
-    path; the results must be bit-identical to an aligned workspace's."""
+    """FFN2's epilogue reads its fp32 residual rows in 32-byte loads when they start on
+    32-byte boundaries and in 16-byte loads otherwise (the out-projection's fp32 output goes
+    out by TMA either way).  A workspace that starts 16 bytes past a 32-byte boundary takes
+    the second path; the results must be bit-identical to an aligned workspace's."""
     shape = synth.LayerShape(1024, 8, 2560)
     H = shape.hidden
     lengths = np.array([96, 160] * 8, np.int32)
